@@ -1,0 +1,77 @@
+"""Partial re-noise and the three-step Euler refinement (oracle side, FP64).
+
+Page: "Open-H3-Regenerate-2K: High-Resolution Video Refinement with
+Few-Step Diffusion" (agientry.com, English article).
+
+* Section "Training: learn what degradation removed": the linear
+  flow-matching path z_sigma = (1 - sigma) z0 + sigma eps with velocity
+  target v = eps - z0.
+* Section "Three steps instead of dozens": the enlarged latent is re-noised
+  to sigma0 = 0.909 by z = (1 - sigma0) z_up + sigma0 eps, then three Euler
+  updates z_{k+1} = z_k + (sigma_{k+1} - sigma_k) v follow the schedule
+  0.909 -> 0.857 -> 0.667 -> 0.
+
+Page "Open-H3-Regenerate-2K-IC" (wujieai.com), section
+"三步接着放大的草稿画，八步从噪声重画": the IC variant starts from
+sigma = 0.835 (up3) or 0.923 (up4) with the same blend.
+
+Reading of the decimals (the pages print decimals only): each sigma is the
+FP32 value nearest to the printed decimal, and both the kernels and this
+oracle use exactly that binary value.  The oracle evaluates every blend in
+FP64 from those exact inputs.
+"""
+
+import numpy as np
+
+# Printed schedule, "Three steps instead of dozens".
+SCHEDULE_DECIMAL = (0.909, 0.857, 0.667, 0.0)
+# IC starts, "三步接着放大的草稿画，八步从噪声重画".
+IC_STARTS_DECIMAL = (0.835, 0.923)
+
+
+def as_fp32(value):
+    """The FP32 value nearest to a printed decimal, as an exact float64."""
+    return float(np.float32(value))
+
+
+SCHEDULE = tuple(as_fp32(s) for s in SCHEDULE_DECIMAL)
+SIGMA0 = SCHEDULE[0]
+
+
+def renoise(up, eps, sigma):
+    """x = (1 - sigma) up + sigma eps, in FP64."""
+    up = np.asarray(up, dtype=np.float64)
+    eps = np.asarray(eps, dtype=np.float64)
+    sigma = float(sigma)
+    return (1.0 - sigma) * up + sigma * eps
+
+
+def euler_step(x, v, sigma, sigma_next):
+    """x + (sigma_next - sigma) v, in FP64."""
+    x = np.asarray(x, dtype=np.float64)
+    v = np.asarray(v, dtype=np.float64)
+    return x + (float(sigma_next) - float(sigma)) * v
+
+
+def flow_point(z0, eps, sigma):
+    """The linear flow path z_sigma = (1 - sigma) z0 + sigma eps (FP64)."""
+    return (1.0 - float(sigma)) * np.asarray(z0, np.float64) + float(sigma) * np.asarray(eps, np.float64)
+
+
+def exact_velocity(z0, eps):
+    """The flow-matching velocity target eps - z0 (FP64)."""
+    return np.asarray(eps, np.float64) - np.asarray(z0, np.float64)
+
+
+def refine(up, eps, schedule, velocity):
+    """Re-noise at schedule[0], then one Euler step per schedule interval.
+
+    velocity(z, k) returns the velocity used at step k.  Returns the list of
+    iterates [z_0, z_1, ..., z_last].
+    """
+    z = renoise(up, eps, schedule[0])
+    out = [z]
+    for k in range(len(schedule) - 1):
+        z = euler_step(z, velocity(z, k), schedule[k], schedule[k + 1])
+        out.append(z)
+    return out

@@ -1,0 +1,89 @@
+"""Pins for the oracle's re-noise and Euler steps.
+
+The pins come from the flow-matching construction on "Open-H3-Regenerate-2K:
+High-Resolution Video Refinement with Few-Step Diffusion": along the linear
+path z_sigma = (1 - sigma) z0 + sigma eps the exact velocity is v = eps - z0,
+so an Euler step from sigma to sigma' lands exactly on z_sigma', and any
+schedule that ends at 0 returns z0 (section "Training: learn what degradation
+removed" for the path, section "Three steps instead of dozens" for the
+re-noise and the schedule).
+"""
+
+import json
+import os
+
+import numpy as np
+import pytest
+
+from oracle import flow
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def _golden(name):
+    with open(os.path.join(GOLDEN, name)) as f:
+        return json.load(f)
+
+
+def test_schedule_constants_match_pages():
+    g = _golden("schedule.json")
+    assert list(flow.SCHEDULE_DECIMAL) == g["sigma_schedule"]
+    assert list(flow.IC_STARTS_DECIMAL) == g["ic_starts"]
+    assert flow.SIGMA0 == float(np.float32(g["sigma0"]))
+    assert flow.SCHEDULE[-1] == 0.0
+
+
+def test_schedule_coefficients_exact_in_fp32():
+    # Sterbenz: for y/2 <= x <= 2y, x - y is exact.  The kernels compute
+    # 1 - sigma and sigma_next - sigma in FP32; they must equal the exact
+    # differences the oracle uses.
+    sig = [np.float32(s) for s in flow.SCHEDULE_DECIMAL]
+    for s in sig + [np.float32(s) for s in flow.IC_STARTS_DECIMAL]:
+        assert float(np.float32(1.0) - s) == 1.0 - float(s)
+    for a, b in zip(sig[:-1], sig[1:]):
+        assert float(b - a) == float(b) - float(a)
+
+
+@pytest.mark.parametrize("start", [0.909, 0.835, 0.923])
+def test_exact_velocity_recovers_z0(start):
+    rng = np.random.default_rng(1)
+    z0 = rng.standard_normal(10000)
+    eps = rng.standard_normal(10000)
+    sched = [flow.as_fp32(start)] + [s for s in flow.SCHEDULE[1:]]
+    if start != 0.909:
+        sched = [flow.as_fp32(start), 0.0]
+    zs = flow.refine(z0, eps, sched, lambda z, k: flow.exact_velocity(z0, eps))
+    # Every iterate sits on the flow path ...
+    for z, s in zip(zs, sched):
+        np.testing.assert_allclose(z, flow.flow_point(z0, eps, s), rtol=0, atol=1e-14)
+    # ... and the last one is z0 (the pages' bound for this check is 1e-5).
+    assert np.abs(zs[-1] - z0).max() < 1e-14
+
+
+def test_three_step_schedule_recovers_z0():
+    rng = np.random.default_rng(2)
+    z0 = rng.standard_normal(5000)
+    eps = rng.standard_normal(5000)
+    zs = flow.refine(z0, eps, flow.SCHEDULE, lambda z, k: flow.exact_velocity(z0, eps))
+    assert len(zs) == 4
+    assert np.abs(zs[-1] - z0).max() < 1e-14
+
+
+def test_renoise_special_cases():
+    rng = np.random.default_rng(3)
+    up = rng.standard_normal(100)
+    eps = rng.standard_normal(100)
+    np.testing.assert_array_equal(flow.renoise(up, eps, 0.0), up)
+    np.testing.assert_array_equal(flow.renoise(up, eps, 1.0), eps)
+    # sigma0 = 0.909 keeps 9.1 % of the draft.
+    x = flow.renoise(up, np.zeros(100), flow.SIGMA0)
+    np.testing.assert_allclose(x, (1.0 - flow.SIGMA0) * up, rtol=1e-15)
+
+
+def test_euler_special_cases():
+    rng = np.random.default_rng(4)
+    x = rng.standard_normal(100)
+    v = rng.standard_normal(100)
+    np.testing.assert_array_equal(flow.euler_step(x, v, 0.5, 0.5), x)
+    # Stepping to sigma' = sigma - 1 adds v with a minus sign.
+    np.testing.assert_allclose(flow.euler_step(x, v, 1.0, 0.0), x - v, rtol=0, atol=1e-15)
