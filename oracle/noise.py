@@ -22,6 +22,11 @@ pair of words (a, b):
 Both are exact in FP32.  Slot 0 / 2 takes rho cos(2 pi u2), slot 1 / 3 takes
 rho sin(2 pi u2).  The oracle evaluates the transform in FP64 and returns the
 unrounded FP64 values; callers round to FP32 where the comparison needs it.
+
+The angle is evaluated as sin/cos of pi t with t = 2 u2 reduced exactly to a
+quarter turn plus a remainder |r| <= 1/4 (t is a dyadic rational, so the
+reduction has no rounding).  Forming 2 pi u2 first would leave a residue of
+order 1e-16 where the exact cosine or sine is 0 (u2 = 1/4, 1/2, 3/4).
 """
 
 import numpy as np
@@ -40,11 +45,30 @@ def uniforms_from_words(a, b):
     return u1, u2
 
 
+def sincos_pi(t):
+    """(sin(pi t), cos(pi t)) in FP64 for dyadic t, with exact argument reduction.
+
+    t = n/2 + r with n = round(2t) and |r| <= 1/4 (exact in FP64 for the
+    dyadic values used here); the quarter-turn identities
+    sin/cos(pi t) = (+-)sin/cos(pi r) then give exact zeros and ones at
+    multiples of 1/2 and full relative accuracy elsewhere.
+    """
+    t = np.asarray(t, dtype=np.float64)
+    n = np.rint(2.0 * t)
+    r = t - 0.5 * n
+    s = np.sin(np.pi * r)
+    c = np.cos(np.pi * r)
+    q = n.astype(np.int64) & 3
+    sin_t = np.select([q == 0, q == 1, q == 2], [s, c, -s], -c)
+    cos_t = np.select([q == 0, q == 1, q == 2], [c, -s, -c], s)
+    return sin_t, cos_t
+
+
 def box_muller(u1, u2):
     """The two deviates (rho cos(2 pi u2), rho sin(2 pi u2)) in FP64."""
     rho = np.sqrt(-2.0 * np.log(u1))
-    theta = 2.0 * np.pi * u2
-    return rho * np.cos(theta), rho * np.sin(theta)
+    sin_t, cos_t = sincos_pi(2.0 * np.asarray(u2, dtype=np.float64))
+    return rho * cos_t, rho * sin_t
 
 
 def normal_from_blocks(words):

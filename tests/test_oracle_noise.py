@@ -31,13 +31,24 @@ def test_u2_zero_puts_radius_on_first_slot():
     assert abs(ea[0] - np.sqrt(48.0 * np.log(2.0))) < 1e-14
 
 
-def test_u2_quarter_puts_radius_on_second_slot():
-    u1, u2 = noise.uniforms_from_words([0x7FFFFF00], [0x40000000])
-    assert u2[0] == 0.25
+def test_quarter_turns_are_exact():
+    # u2 = 1/4, 1/2, 3/4: the pair is (0, rho), (-rho, 0), (0, -rho) exactly.
+    a = [0x7FFFFF00] * 3
+    u1, u2 = noise.uniforms_from_words(a, [0x40000000, 0x80000000, 0xC0000000])
+    assert u2.tolist() == [0.25, 0.5, 0.75]
     ea, eb = noise.box_muller(u1, u2)
     rho = np.sqrt(-2.0 * np.log(u1[0]))
-    assert abs(ea[0]) < 1e-15 * max(rho, 1.0)
-    assert abs(eb[0] - rho) < 1e-15 * rho
+    assert ea.tolist() == [0.0, -rho, 0.0]
+    assert eb.tolist() == [rho, 0.0, -rho]
+
+
+def test_angle_matches_plain_trig_away_from_quarter_turns():
+    rng = np.random.default_rng(1)
+    u2 = rng.integers(0, 2**24, size=100000).astype(np.float64) * 2.0 ** -24
+    s, c = noise.sincos_pi(2.0 * u2)
+    # The plain formula itself is off by up to ~ulp(2 pi) from rounding 2 pi u2.
+    np.testing.assert_allclose(s, np.sin(2.0 * np.pi * u2), rtol=0, atol=1e-15)
+    np.testing.assert_allclose(c, np.cos(2.0 * np.pi * u2), rtol=0, atol=1e-15)
 
 
 def test_low_byte_of_words_is_ignored():
