@@ -1,0 +1,583 @@
+"""Benchmark of the merged-LoRA refiner hot path on B200.
+
+One step is one pass of the whole path over the 2K workload (latent
+37 x 24 x 90 x 160, 532,800 tokens, d = 7168, merged rank 576):
+
+  lora_merge for the three layer shapes (d->d, d->3d, 4d->d)
+  renoise(up) at sigma0 = 0.909
+  lora_linear d->d,   euler_step 0.909 -> 0.857
+  lora_linear d->3d,  euler_step 0.857 -> 0.667
+  lora_linear 4d->d,  euler_step 0.667 -> 0
+
+(each Euler step follows one stand-in transformer pass, as in the refine
+loop).  `value` is tokens/s over the whole job (tokens of every rank divided
+by the slowest rank's time); with N GPUs each rank runs its own copy of the
+workload (weak scaling, no data-path collective).
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+`--impl reference` times the FP64 CPU oracle on the host cores over a
+bounded sample of tokens per step (the reference arm for this path).
+"""
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "lora_linear tokens/s + % bf16 TC peak at 2K grid; renoise/Euler HBM GB/s"
+UNIT = "tokens/s"
+WORKLOAD = "2k"
+FALLBACK_HBM_GBS = 6650.0
+FALLBACK_BF16_TFLOPS = 1590.0
+FALLBACK_BF16_TFLOPS_SUSTAINED = 1400.0
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        return {
+            "hbm_gbs": float(p["hbm_gbs"]),
+            "bf16_tflops": float(p["bf16_tflops"]),
+            "bf16_tflops_sustained": float(p.get("bf16_tflops_sustained", p["bf16_tflops"])),
+            "source": "measured",
+        }
+    except (OSError, KeyError, ValueError):
+        return {
+            "hbm_gbs": FALLBACK_HBM_GBS,
+            "bf16_tflops": FALLBACK_BF16_TFLOPS,
+            "bf16_tflops_sustained": FALLBACK_BF16_TFLOPS_SUSTAINED,
+            "source": "fallback",
+        }
+
+
+# ---------------------------------------------------------------------------
+# Distributed plumbing (one process per GPU; NCCL only for barrier / max).
+# ---------------------------------------------------------------------------
+def dist_setup(n_gpus):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world != n_gpus:
+        raise SystemExit(f"--gpus {n_gpus} but WORLD_SIZE={world}")
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=600),
+                                device_id=torch.device("cuda", local))
+    else:
+        torch.cuda.set_device(0)
+    return rank, world, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+
+        dist.barrier()
+
+
+def max_over_ranks(value, world):
+    if world == 1:
+        return value
+    import torch.distributed as dist
+
+    t = torch.tensor([value], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+# ---------------------------------------------------------------------------
+# Clock sampling during the timed region.
+# ---------------------------------------------------------------------------
+class ClockSampler:
+    QUERY = ("index,uuid,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index):
+        self.proc = None
+        self.path = None
+        try:
+            uuid = torch.cuda.get_device_properties(device_index).uuid
+            self.uuid = "GPU-" + str(uuid) if not str(uuid).startswith("GPU-") else str(uuid)
+        except Exception:
+            self.uuid = None
+
+    def start(self):
+        fd, self.path = tempfile.mkstemp(suffix=".csv")
+        os.close(fd)
+        cmd = ["nvidia-smi", f"--query-gpu={self.QUERY}", "--format=csv,noheader,nounits", "-lms", "200"]
+        if self.uuid:
+            cmd += ["-i", self.uuid]
+        try:
+            self.out = open(self.path, "w")
+            self.proc = subprocess.Popen(cmd, stdout=self.out, stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.out.close()
+        rows = []
+        with open(self.path) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) >= 10:
+                    rows.append(parts)
+        os.unlink(self.path)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+
+        def num(s):
+            try:
+                return float(s)
+            except ValueError:
+                return None
+
+        sm = [num(r[2]) for r in rows if num(r[2]) is not None]
+        mx = [num(r[3]) for r in rows if num(r[3]) is not None]
+        reasons = set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for r in rows:
+            for name, val in zip(names, r[6:10]):
+                if val.strip().lower() == "active":
+                    reasons.add(name)
+        return {
+            "sm_mhz": statistics.median(sm) if sm else None,
+            "sm_max_mhz": max(mx) if mx else None,
+            "reasons": sorted(reasons),
+            "samples": len(rows),
+            "power_w_max": max((num(r[4]) or 0.0) for r in rows),
+        }
+
+
+# ---------------------------------------------------------------------------
+# Our arm.
+# ---------------------------------------------------------------------------
+def layer_flops(M, K, N, R):
+    return 2.0 * M * (K * N + K * R + R * N)
+
+
+class Problem:
+    """Device-resident inputs and outputs of one 2K step."""
+
+    def __init__(self, w, dev):
+        from lora_gemm_b200 import synth
+        import lora_gemm_b200 as lg
+
+        self.w = w
+        M = w.tokens
+        R = sum(synth.ADAPTER_RANKS)
+        self.R = R
+        self.layers = []
+        x_by_k = {}
+        for i, (K, N) in enumerate(w.shapes):
+            if K not in x_by_k:
+                x_by_k[K] = synth.activations(w, K, i, dev)
+            As, Bs = synth.adapters(w, i, dev)
+            L = {
+                "K": K, "N": N, "x": x_by_k[K], "W": synth.weight(w, i, dev), "As": As, "Bs": Bs,
+                "A_cat": torch.empty((R, K), dtype=torch.float32, device=dev),
+                "B_cat": torch.empty((N, R), dtype=torch.float32, device=dev),
+                "y": torch.empty((M, N), dtype=torch.bfloat16, device=dev),
+                "ws": torch.empty(lg.lora_linear_workspace_size(M, K, N, R), dtype=torch.uint8, device=dev),
+            }
+            self.layers.append(L)
+        self.up = synth.upscaled_latent(w, dev)
+        self.x_lat = torch.empty_like(self.up)
+        self.v = [synth.velocity(w, k, dev) for k in range(3)]
+        self.sigmas = [float(torch.tensor(s, dtype=torch.float32)) for s in synth.SIGMA_SCHEDULE]
+        self.scales = synth.ADAPTER_SCALES
+
+
+def run_step(P, ev=None):
+    """One pass of the hot path on the current stream; ev collects (name, start, end) event pairs."""
+    import lora_gemm_b200 as lg
+
+    def rec(name, fn):
+        if ev is None:
+            fn()
+            return
+        s = torch.cuda.Event(enable_timing=True)
+        e = torch.cuda.Event(enable_timing=True)
+        s.record()
+        fn()
+        e.record()
+        ev.append((name, s, e))
+
+    for L in P.layers:
+        rec("lora_merge", lambda L=L: lg.lora_merge(L["As"], L["Bs"], P.scales, L["A_cat"], L["B_cat"]))
+    rec("renoise", lambda: lg.renoise(P.up, P.sigmas[0], P.w.seed, out=P.x_lat))
+    for k, L in enumerate(P.layers):
+        rec(f"lora_linear{k}", lambda L=L: lg.lora_linear(L["x"], L["W"], L["A_cat"], L["B_cat"], y=L["y"],
+                                                          workspace=L["ws"]))
+        rec(f"euler{k}", lambda k=k: lg.euler_step(P.x_lat, P.v[k], P.sigmas[k], P.sigmas[k + 1]))
+
+
+def bytes_per_kernel(P):
+    w = P.w
+    n = w.latent_numel
+    M = w.tokens
+    merge = sum(4 * P.R * (L["K"] + L["N"]) * 2 for L in P.layers)  # read adapters, write merged
+    return {"renoise": 8.0 * n, "euler": 12.0 * n, "lora_merge": merge / len(P.layers),
+            "lora_linear_min_bytes": [2.0 * (M * L["K"] + L["N"] * L["K"] + M * L["N"]) + 4.0 * P.R * (L["K"] + L["N"])
+                                      for L in P.layers]}
+
+
+def run_ours(args, rank, world, local):
+    import lora_gemm_b200 as lg
+    from lora_gemm_b200 import synth
+
+    peaks = load_peaks()
+    dev = torch.device("cuda", torch.cuda.current_device())
+    w = synth.WORKLOADS[args.workload]
+    P = Problem(w, dev)
+    torch.cuda.synchronize()
+
+    for _ in range(args.warmup):
+        run_step(P)
+    torch.cuda.synchronize()
+    if lg.get_last_device_error() != lg.LG_OK:
+        raise SystemExit("device error during warm-up")
+
+    clocks = ClockSampler(dev.index) if rank == 0 else None
+    if clocks:
+        clocks.start()
+    ev = []
+    launches0 = lg.launch_count()
+    barrier(world)
+    torch.cuda.synchronize()
+    t_start = torch.cuda.Event(enable_timing=True)
+    t_end = torch.cuda.Event(enable_timing=True)
+    t_start.record()
+    for _ in range(args.steps):
+        run_step(P, ev)
+    t_end.record()
+    torch.cuda.synchronize()
+    barrier(world)
+    launches = lg.launch_count() - launches0
+    clk = clocks.stop() if clocks else None
+    status = lg.get_last_device_error()
+    if status != lg.LG_OK:
+        raise SystemExit(f"device error during timed steps: {lg.status_string(status)}")
+
+    elapsed_ms = t_start.elapsed_time(t_end)
+    elapsed_ms = max_over_ranks(elapsed_ms, world)
+    per = {}
+    for name, s, e in ev:
+        per.setdefault(name, []).append(s.elapsed_time(e))
+    M = w.tokens
+    value = world * M * args.steps / (elapsed_ms * 1e-3)
+
+    # Dominant kernel: lora_linear (tensor-bound).
+    flops = [layer_flops(M, L["K"], L["N"], P.R) for L in P.layers]
+    lin_ms = [statistics.mean(per[f"lora_linear{k}"]) for k in range(len(P.layers))]
+    achieved_tflops = sum(flops) / (sum(lin_ms) * 1e-3) / 1e12
+    peak_t = peaks["bf16_tflops_sustained"]
+    traffic = load_traffic()
+    bpk = bytes_per_kernel(P)
+    ren_ms = statistics.mean(per["renoise"])
+    eul_ms = statistics.mean([t for k in range(3) for t in per[f"euler{k}"]])
+    mer_ms = statistics.mean(per["lora_merge"])
+    hbm = peaks["hbm_gbs"]
+
+    def gbs(b, ms):
+        return b / (ms * 1e-3) / 1e9
+
+    kernels = {
+        "lora_linear": {
+            "per_layer_ms": [round(t, 4) for t in lin_ms],
+            "per_layer_tflops": [round(f / (t * 1e-3) / 1e12, 1) for f, t in zip(flops, lin_ms)],
+            "tflops": round(achieved_tflops, 1),
+            "frac_of_measured_sustained": round(achieved_tflops / peak_t, 4),
+            "frac_of_measured_burst": round(achieved_tflops / peaks["bf16_tflops"], 4),
+            "frac_of_spec_2250": round(achieved_tflops / 2250.0, 4),
+            "tokens_per_s_per_layer": [round(M / (t * 1e-3), 1) for t in lin_ms],
+            "note": "time includes the bf16 conversion of the merged factors inside the call",
+        },
+        "renoise": {"ms": round(ren_ms, 5), "gbs": round(gbs(bpk["renoise"], ren_ms), 1),
+                    "frac_of_measured_hbm": round(gbs(bpk["renoise"], ren_ms) / hbm, 4),
+                    "frac_of_8000": round(gbs(bpk["renoise"], ren_ms) / 8000.0, 4)},
+        "euler_step": {"ms": round(eul_ms, 5), "gbs": round(gbs(bpk["euler"], eul_ms), 1),
+                       "frac_of_measured_hbm": round(gbs(bpk["euler"], eul_ms) / hbm, 4),
+                       "frac_of_8000": round(gbs(bpk["euler"], eul_ms) / 8000.0, 4)},
+        "lora_merge": {"ms": round(mer_ms, 5), "gbs": round(gbs(bpk["lora_merge"], mer_ms), 1)},
+    }
+    result = {
+        "metric": METRIC,
+        "value": round(value, 1),
+        "unit": UNIT,
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": round(elapsed_ms / args.steps, 3),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16",
+        "dtype_detail": "bf16 x, W and factor copies on the tensor cores with FP32 accumulate; FP32 latent",
+        "data": "synthetic (seeded torch draws shaped like the pages' 2K grid; no weights)",
+        "config": {
+            "workload": w.name,
+            "latent": list(w.latent_shape),
+            "tokens": M,
+            "d": w.d,
+            "layers_k_n": [list(s) for s in w.shapes],
+            "rank": P.R,
+            "adapter_ranks": list(synth.ADAPTER_RANKS),
+            "schedule": list(synth.SIGMA_SCHEDULE),
+            "parallelism": f"replicas x{world} (weak scaling, no collective)",
+            "l2": "no explicit flush: lora_linear inputs (7.6-30.5 GB) exceed L2, and each elementwise kernel's "
+                  "inputs were last touched before >= 364 MB of other traffic",
+        },
+        "roofline": {
+            "bound": "tensor",
+            "kernel": "k_lora_linear",
+            "achieved": round(achieved_tflops, 1),
+            "peak": peak_t,
+            "peak_kind": f"bf16_tflops_sustained ({peaks['source']})",
+            "unit": "TFLOP/s",
+            "frac": round(achieved_tflops / peak_t, 4),
+            "traffic": traffic,
+            "algorithmic_flops_per_token": sum(f / M for f in flops),
+        },
+        "kernels": kernels,
+        "clocks": clk,
+        "gpu_launches": int(launches),
+        "launches_per_step": int(launches) // max(args.steps, 1),
+    }
+    if not args.no_e2e:
+        result["e2e"] = run_e2e(P, args, world)
+    if rank == 0 and not args.no_cpu_baseline:
+        result["cpu_baseline"] = cpu_baseline(w, target_s=args.cpu_seconds)
+    return result
+
+
+def load_traffic():
+    """DRAM bytes per lora_linear launch from the committed ncu summary, if current."""
+    path = os.path.join(ROOT, "profiles", "lora_linear_traffic.json")
+    try:
+        with open(path) as f:
+            t = json.load(f)
+        return t.get("traffic_bytes_per_launch")
+    except (OSError, ValueError):
+        return None
+
+
+def run_e2e(P, args, world):
+    """Same step through the public API with host buffers: H2D of the step's
+    inputs (activations, latent, velocities) from pinned memory, the step,
+    D2H of its results (y of each layer, the final latent), all timed."""
+    host_in = {}
+    host_out = {}
+    seen = set()
+    for L in P.layers:
+        if id(L["x"]) not in seen:
+            seen.add(id(L["x"]))
+            host_in[id(L["x"])] = (L["x"], torch.empty(L["x"].shape, dtype=L["x"].dtype, pin_memory=True))
+        host_out[id(L["y"])] = (L["y"], torch.empty(L["y"].shape, dtype=L["y"].dtype, pin_memory=True))
+    for t in [P.up] + P.v:
+        host_in[id(t)] = (t, torch.empty(t.shape, dtype=t.dtype, pin_memory=True))
+    host_out[id(P.x_lat)] = (P.x_lat, torch.empty(P.x_lat.shape, dtype=P.x_lat.dtype, pin_memory=True))
+    for dev_t, host_t in host_in.values():
+        host_t.copy_(dev_t)
+    h2d = sum(d.numel() * d.element_size() for d, _ in host_in.values())
+    d2h = sum(d.numel() * d.element_size() for d, _ in host_out.values())
+
+    def step():
+        for dev_t, host_t in host_in.values():
+            dev_t.copy_(host_t, non_blocking=True)
+        run_step(P)
+        for dev_t, host_t in host_out.values():
+            host_t.copy_(dev_t, non_blocking=True)
+
+    step()
+    torch.cuda.synchronize()
+    steps = max(1, min(args.steps, 3))
+    barrier(world)
+    torch.cuda.synchronize()
+    s = torch.cuda.Event(enable_timing=True)
+    e = torch.cuda.Event(enable_timing=True)
+    s.record()
+    for _ in range(steps):
+        step()
+    e.record()
+    torch.cuda.synchronize()
+    barrier(world)
+    ms = max_over_ranks(s.elapsed_time(e), world)
+    return {"value": round(world * P.w.tokens * steps / (ms * 1e-3), 1), "unit": UNIT,
+            "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h), "steps": steps,
+            "ms_per_step": round(ms / steps, 3)}
+
+
+# ---------------------------------------------------------------------------
+# The FP64 oracle on the host cores.
+# ---------------------------------------------------------------------------
+def blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+
+        info = threadpool_info()
+        n = [d.get("num_threads", 1) for d in info if d.get("user_api") == "blas"]
+        return max(n) if n else 1
+    except Exception:
+        return os.cpu_count() or 1
+
+
+class OracleStep:
+    """The whole path for a sample of `tokens` tokens of the workload, in FP64 on the CPU."""
+
+    def __init__(self, w, tokens):
+        import numpy as np
+
+        from lora_gemm_b200 import synth
+
+        self.w = w
+        self.tokens = tokens
+        self.np = np
+        g = np.random.default_rng(w.seed)
+        self.layers = []
+        for K, N in w.shapes:
+            x = g.standard_normal((tokens, K)).astype(np.float32).astype(np.float64)
+            W = g.standard_normal((N, K)) * K ** -0.5
+            As = [(g.standard_normal((r, K)) * K ** -0.5).astype(np.float32) for r in synth.ADAPTER_RANKS]
+            Bs = [(g.standard_normal((N, r)) * synth.B_STD).astype(np.float32) for r in synth.ADAPTER_RANKS]
+            self.layers.append((x, W, As, Bs))
+        n = tokens * w.channels
+        self.n = n
+        self.up = g.standard_normal(n).astype(np.float32)
+        self.v = [g.standard_normal(n).astype(np.float32) for _ in range(3)]
+        self.scales = synth.ADAPTER_SCALES
+
+    def run(self):
+        from oracle import flow, lora, noise
+
+        eps = noise.normal(self.w.seed, 0, self.n)
+        z = flow.renoise(self.up, eps, flow.SCHEDULE[0])
+        for k, (x, W, As, Bs) in enumerate(self.layers):
+            A_cat, B_cat = lora.lora_merge(As, Bs, self.scales)
+            lora.lora_linear(x, W, A_cat, B_cat)
+            z = flow.euler_step(z, self.v[k], flow.SCHEDULE[k], flow.SCHEDULE[k + 1])
+        return z
+
+
+def cpu_baseline(w, target_s=15.0):
+    probe = OracleStep(w, 32)
+    probe.run()
+    t0 = time.perf_counter()
+    probe.run()
+    t_probe = time.perf_counter() - t0
+    tokens = int(max(32, min(4096, 32 * target_s / max(t_probe, 1e-3))))
+    step = OracleStep(w, tokens)
+    t0 = time.perf_counter()
+    step.run()
+    dt = time.perf_counter() - t0
+    return {"value": round(tokens / dt, 2), "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
+            "sample": f"{tokens} tokens of the {w.name} workload through merge, renoise, the three layers and "
+                      f"three Euler steps in FP64 ({dt:.1f} s)"}
+
+
+def run_reference(args, rank, world):
+    from lora_gemm_b200 import synth
+
+    w = synth.WORKLOADS[args.workload]
+    probe = OracleStep(w, 32)
+    probe.run()
+    t0 = time.perf_counter()
+    probe.run()
+    t_probe = time.perf_counter() - t0
+    per_step_s = 90.0 / max(1, args.steps + args.warmup)
+    tokens = int(max(32, min(2048, 32 * per_step_s / max(t_probe, 1e-3))))
+    step = OracleStep(w, tokens)
+    for _ in range(args.warmup):
+        step.run()
+    times = []
+    for _ in range(args.steps):
+        t0 = time.perf_counter()
+        step.run()
+        times.append(time.perf_counter() - t0)
+    total = sum(times)
+    value = tokens * args.steps / total
+    sample = (f"{tokens} tokens of the {w.name} workload per step through merge, renoise, the three layers "
+              f"and three Euler steps in FP64 on the host CPU")
+    return {
+        "impl": "reference",
+        "metric": METRIC,
+        "value": round(value, 2),
+        "unit": UNIT,
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": round(1e3 * total / args.steps, 3),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "f64",
+        "data": "synthetic",
+        "config": {"workload": w.name, "latent": list(w.latent_shape), "tokens": w.tokens, "d": w.d,
+                   "layers_k_n": [list(s) for s in w.shapes], "rank": sum(synth.ADAPTER_RANKS),
+                   "parallelism": "host CPU (rank 0 only)"},
+        "cpu_baseline": {"value": round(value, 2), "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": round(value, 2), "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=5)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default=WORKLOAD)
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    args = ap.parse_args()
+    if args.warmup < 3:
+        raise SystemExit("--warmup must be >= 3")
+
+    if args.impl == "reference":
+        rank = int(os.environ.get("RANK", "0"))
+        world = int(os.environ.get("WORLD_SIZE", "1"))
+        if rank != 0:
+            return
+        print(json.dumps(run_reference(args, rank, world)), flush=True)
+        return
+
+    rank, world, local = dist_setup(args.gpus)
+    try:
+        result = run_ours(args, rank, world, local)
+        if rank == 0:
+            print(json.dumps(result), flush=True)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,199 @@
+/*
+ * lora_gemm.h -- C ABI of the B200 (sm_100a) merged-LoRA refiner hot path.
+ *
+ * The operations come from the Open-H3-Regenerate-2K pages:
+ *
+ *   lg_lora_merge   "Open-H3-Regenerate-2K：MiniMax H3 的开源 4K 精修方案"
+ *                   (comfyui-wiki.com news), section "三个步如何完成工作":
+ *                   adapters merged by concatenating factors along the rank
+ *                   axis (384 + 128 + 64 = 576), stored in FP32.
+ *   lg_lora_linear  the frozen transformer's linear layer carrying that merged
+ *                   LoRA ("Open-H3-Regenerate-2K: High-Resolution Video
+ *                   Refinement with Few-Step Diffusion", section "The
+ *                   four-stage refinement pipeline"):
+ *                   y = x W^T + (x A_cat^T) B_cat^T.
+ *   lg_renoise      same page, section "Three steps instead of dozens":
+ *                   z = (1 - sigma0) z_up + sigma0 eps, eps ~ N(0, I).
+ *   lg_euler_step   same section: z_{k+1} = z_k + (sigma_{k+1} - sigma_k) v on
+ *                   the schedule 0.909 -> 0.857 -> 0.667 -> 0.
+ *
+ * The pages name no random number generator.  This library draws eps from a
+ * Philox4x32-10 stream (Salmon et al., "Parallel Random Numbers: As Easy as
+ * 1, 2, 3", SC'11) with key = (seed mod 2^32, seed >> 32) and counter
+ * (j mod 2^32, j >> 32, 0, 0) for 4-element block j, turned into normals by
+ * the Box-Muller transform (see lg_philox_normal).
+ *
+ * Conventions for every entry point:
+ *   - All tensor pointers are DEVICE pointers on the current CUDA device,
+ *     owned by the caller.  The library allocates no device memory; the
+ *     scratch that lg_lora_linear needs is the caller's workspace.
+ *   - `stream` is a cudaStream_t passed as void* (NULL = legacy default
+ *     stream).  Calls are asynchronous on that stream.  The return value
+ *     reports argument validation and launch errors only; a device-side
+ *     timeout is reported later by lg_get_last_device_error().
+ *   - Arguments are validated before anything is launched; on any error
+ *     nothing is launched and nothing is written.
+ *   - Kernels are compiled for sm_100a only; on another device every compute
+ *     entry point returns LG_ERR_NOT_SM100.
+ *   - Element counts of zero are valid and launch nothing.
+ */
+#ifndef LORA_GEMM_H
+#define LORA_GEMM_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum lg_status {
+  LG_OK = 0,
+  LG_ERR_INVALID_ARG = 1,       /* null pointer, negative size, bad sigma, ... */
+  LG_ERR_UNSUPPORTED_SHAPE = 2, /* a dimension outside the supported set */
+  LG_ERR_MISALIGNED = 3,        /* a pointer not aligned as documented */
+  LG_ERR_WORKSPACE = 4,         /* workspace missing or too small */
+  LG_ERR_CUDA = 5,              /* a CUDA runtime/driver call failed */
+  LG_ERR_DEVICE_TIMEOUT = 6,    /* a bounded wait inside a kernel ran out */
+  LG_ERR_NOT_SM100 = 7          /* current device is not compute capability 10.0 */
+} lg_status;
+
+/* Short English description of a status code (static storage). */
+const char* lg_status_string(int status);
+
+/* Library version as 10000*major + 100*minor + patch. */
+int lg_version(void);
+
+/* Number of kernels this library has launched in this process (all devices).
+ * A monotone counter; callers take differences around a region of interest. */
+uint64_t lg_launch_count(void);
+
+/* Synchronizes `stream`, then reads and clears the current device's error
+ * word.  Returns LG_OK if no kernel recorded an error since the last call,
+ * LG_ERR_DEVICE_TIMEOUT if a bounded wait in a kernel gave up (the kernel
+ * then abandoned its work, drained its own copies, freed its tensor memory
+ * and returned; its outputs are undefined), or LG_ERR_CUDA if the
+ * synchronization itself failed. */
+lg_status lg_get_last_device_error(void* stream);
+
+/* Upper bound, in nanoseconds, on any single wait inside lg_lora_linear's
+ * pipeline (default 4e9).  Process-wide; applies to launches made after the
+ * call.  0 restores the default.  Meant for fault-injection tests: a tiny
+ * limit makes the waits run out so the timeout path can be exercised. */
+void lg_set_wait_limit_ns(uint64_t limit_ns);
+
+/* ------------------------------------------------------------------------
+ * lg_lora_merge -- concatenate n_adapters LoRA adapters along the rank axis.
+ *
+ *   A_cat[off_i + r][k] = scales[i] * A[i][r][k]      (FP32, one rounding)
+ *   B_cat[o][off_i + r] = B[i][o][r]                  (FP32, exact copy)
+ *
+ * with off_i = ranks[0] + ... + ranks[i-1] and R = sum of ranks, so that
+ * B_cat A_cat = sum_i scales[i] B_i A_i.  The scale sits on A (the pages do
+ * not say which factor carries it).
+ *
+ *   A, B        HOST arrays of n_adapters DEVICE pointers.  A[i] is row-major
+ *               [ranks[i], d_in] FP32; B[i] is row-major [d_out, ranks[i]].
+ *   ranks       HOST array, each >= 1 and a multiple of 4.
+ *   scales      HOST array of n_adapters FP32 scales.
+ *   A_cat       DEVICE [R, d_in] FP32 row-major (output).
+ *   B_cat       DEVICE [d_out, R] FP32 row-major (output).
+ *   1 <= n_adapters <= 8; d_in, d_out >= 1 and multiples of 4; all device
+ *   pointers 16-byte aligned (else LG_ERR_MISALIGNED).  Outputs must not
+ *   overlap inputs.
+ * ---------------------------------------------------------------------- */
+lg_status lg_lora_merge(int n_adapters, const float* const* A, const float* const* B,
+                        const int* ranks, const float* scales, int d_in, int d_out,
+                        float* A_cat, float* B_cat, void* stream);
+
+/* Bytes of workspace lg_lora_linear needs for this shape (bf16 copies of the
+ * merged factors, each padded to 256 bytes).  Returns 0 when no workspace is
+ * needed (R = 0) or the shape is unsupported (lg_lora_linear then says
+ * which argument is wrong). */
+size_t lg_lora_linear_workspace_size(int64_t M, int K, int N, int R);
+
+/* ------------------------------------------------------------------------
+ * lg_lora_linear -- merged-LoRA linear layer over latent tokens:
+ *
+ *   y = x W^T + (x A_cat^T) B_cat^T
+ *
+ *   x      DEVICE [M, K] bf16 row-major (token activations).
+ *   W      DEVICE [N, K] bf16 row-major (frozen weight, y = x W^T).
+ *   A_cat  DEVICE [R, K] FP32 row-major (merged down-projection factor).
+ *   B_cat  DEVICE [N, R] FP32 row-major (merged up-projection factor).
+ *   y      DEVICE [M, N] bf16 row-major (output, round-to-nearest-even).
+ *   workspace, ws_bytes  DEVICE scratch of at least
+ *          lg_lora_linear_workspace_size(M, K, N, R) bytes; contents on
+ *          entry are ignored and clobbered.
+ *
+ * Arithmetic: the FP32 factors are rounded to bf16 (RNE) for the tensor
+ * cores; all products accumulate in FP32; the rank-R intermediate
+ * h = x A_cat^T is rounded to bf16 and kept on chip (tensor memory), never
+ * written to global memory.
+ *
+ * Shapes: M >= 0 (0 launches nothing; M < 2^31); K a multiple of 64 and
+ * >= 64; N a multiple of 32 and >= 32; R a multiple of 64 with
+ * 0 <= R <= 576 (R = 0: plain GEMM, A_cat and B_cat may be NULL).  All
+ * pointers 16-byte aligned.  y must not overlap x, W, A_cat, B_cat or the
+ * workspace.
+ * ---------------------------------------------------------------------- */
+lg_status lg_lora_linear(const void* x, const void* W, const float* A_cat, const float* B_cat,
+                         void* y, int64_t M, int K, int N, int R,
+                         void* workspace, size_t ws_bytes, void* stream);
+
+/* ------------------------------------------------------------------------
+ * lg_renoise -- partial re-noise of an upscaled latent:
+ *
+ *   x[i] = (1 - sigma) * up[i] + sigma * eps[offset + i],  i in [0, n)
+ *
+ * eps[e] is element e of the Philox/Box-Muller stream for `seed` (see
+ * lg_philox_normal).  The blend is evaluated from the unrounded eps and
+ * rounded once to FP32.
+ *
+ *   up, x   DEVICE FP32 arrays of n elements (flat [F, C, H, W] latent);
+ *           x == up (in place) is allowed, partial overlap is not.
+ *   sigma   0 <= sigma <= 1.
+ *   offset  flat index of up[0] in the global latent; a multiple of 4.
+ *   Pointers 16-byte aligned.
+ * ---------------------------------------------------------------------- */
+lg_status lg_renoise(const float* up, float* x, int64_t n, float sigma, uint64_t seed,
+                     uint64_t offset, void* stream);
+
+/* ------------------------------------------------------------------------
+ * lg_euler_step -- one flow-matching Euler step, in place:
+ *
+ *   x[i] = x[i] + (sigma_next - sigma) * v[i]
+ *
+ * computed as fmaf(sigma_next - sigma, v[i], x[i]) with the difference taken
+ * in FP32 (exact for the schedule 0.909 -> 0.857 -> 0.667 -> 0 by
+ * Sterbenz's lemma).
+ *
+ *   x, v    DEVICE FP32 arrays of n elements; must not overlap.
+ *   Pointers 16-byte aligned; sigma, sigma_next finite.
+ * ---------------------------------------------------------------------- */
+lg_status lg_euler_step(float* x, const float* v, int64_t n, float sigma, float sigma_next,
+                        void* stream);
+
+/* ------------------------------------------------------------------------
+ * Generator hooks (same generator as lg_renoise), for testing.
+ *
+ * lg_philox_u32: out[4b + t] = word t of Philox4x32-10(counter of block
+ *   block_offset + b, key of seed), b in [0, n_blocks).  out: DEVICE uint32,
+ *   4 * n_blocks words, 16-byte aligned.
+ *
+ * lg_philox_normal: eps[i] = FP32 rounding of element offset + i of the
+ *   normal stream.  Element e uses block j = e / 4, slot t = e % 4; words
+ *   (a, b) = (r0, r1) for slots 0-1 and (r2, r3) for slots 2-3;
+ *   u1 = ((a >> 8) + 1) 2^-24, u2 = (b >> 8) 2^-24; slot 0/2 is
+ *   sqrt(-2 ln u1) cos(2 pi u2), slot 1/3 is sqrt(-2 ln u1) sin(2 pi u2).
+ *   eps: DEVICE FP32, n elements, 16-byte aligned; offset a multiple of 4.
+ * ---------------------------------------------------------------------- */
+lg_status lg_philox_u32(uint32_t* out, int64_t n_blocks, uint64_t seed, uint64_t block_offset,
+                        void* stream);
+lg_status lg_philox_normal(float* eps, int64_t n, uint64_t seed, uint64_t offset, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* LORA_GEMM_H */

@@ -1,0 +1,253 @@
+"""Thin Python binding of the lora_gemm C ABI (include/lora_gemm.h).
+
+Every function here only marshals arguments -- checks dtypes, shapes,
+devices and contiguity of torch tensors, allocates outputs with torch when
+the caller does not pass them, and hands raw device pointers plus the current
+CUDA stream to liblora_gemm.so.  All arithmetic runs in the library's CUDA
+kernels; there is no CPU path.  Importing this package fails with ImportError
+when the compiled library is missing (build it with
+``python -m lora_gemm_b200.build``).
+"""
+
+import ctypes
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "liblora_gemm.so")
+
+LG_OK = 0
+LG_ERR_INVALID_ARG = 1
+LG_ERR_UNSUPPORTED_SHAPE = 2
+LG_ERR_MISALIGNED = 3
+LG_ERR_WORKSPACE = 4
+LG_ERR_CUDA = 5
+LG_ERR_DEVICE_TIMEOUT = 6
+LG_ERR_NOT_SM100 = 7
+
+# Exported C symbols and their ctypes signatures (the header's declarations).
+_c_void_p = ctypes.c_void_p
+_SIGNATURES = {
+    "lg_status_string": (ctypes.c_char_p, [ctypes.c_int]),
+    "lg_version": (ctypes.c_int, []),
+    "lg_launch_count": (ctypes.c_uint64, []),
+    "lg_get_last_device_error": (ctypes.c_int, [_c_void_p]),
+    "lg_set_wait_limit_ns": (None, [ctypes.c_uint64]),
+    "lg_lora_merge": (
+        ctypes.c_int,
+        [ctypes.c_int, ctypes.POINTER(_c_void_p), ctypes.POINTER(_c_void_p), ctypes.POINTER(ctypes.c_int),
+         ctypes.POINTER(ctypes.c_float), ctypes.c_int, ctypes.c_int, _c_void_p, _c_void_p, _c_void_p],
+    ),
+    "lg_lora_linear_workspace_size": (ctypes.c_size_t, [ctypes.c_int64, ctypes.c_int, ctypes.c_int, ctypes.c_int]),
+    "lg_lora_linear": (
+        ctypes.c_int,
+        [_c_void_p, _c_void_p, _c_void_p, _c_void_p, _c_void_p, ctypes.c_int64, ctypes.c_int, ctypes.c_int,
+         ctypes.c_int, _c_void_p, ctypes.c_size_t, _c_void_p],
+    ),
+    "lg_renoise": (
+        ctypes.c_int,
+        [_c_void_p, _c_void_p, ctypes.c_int64, ctypes.c_float, ctypes.c_uint64, ctypes.c_uint64, _c_void_p],
+    ),
+    "lg_euler_step": (
+        ctypes.c_int, [_c_void_p, _c_void_p, ctypes.c_int64, ctypes.c_float, ctypes.c_float, _c_void_p]
+    ),
+    "lg_philox_u32": (ctypes.c_int, [_c_void_p, ctypes.c_int64, ctypes.c_uint64, ctypes.c_uint64, _c_void_p]),
+    "lg_philox_normal": (ctypes.c_int, [_c_void_p, ctypes.c_int64, ctypes.c_uint64, ctypes.c_uint64, _c_void_p]),
+}
+EXPORTED_SYMBOLS = tuple(_SIGNATURES)
+
+
+def _load():
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(
+            f"lora_gemm CUDA library not found at {LIB_PATH}; build it with `python -m lora_gemm_b200.build`"
+        )
+    lib = ctypes.CDLL(LIB_PATH)
+    for name, (res, args) in _SIGNATURES.items():
+        fn = getattr(lib, name)
+        fn.restype = res
+        fn.argtypes = args
+    return lib
+
+
+lib = _load()
+
+
+class LoraGemmError(RuntimeError):
+    def __init__(self, status, where):
+        self.status = status
+        msg = lib.lg_status_string(status).decode()
+        super().__init__(f"{where}: status {status} ({msg})")
+
+
+def _check(status, where):
+    if status != LG_OK:
+        raise LoraGemmError(status, where)
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(device):
+    return ctypes.c_void_p(torch.cuda.current_stream(device).cuda_stream)
+
+
+def _need(t, dtype, name, ndim=None):
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if ndim is not None and t.dim() != ndim:
+        raise ValueError(f"{name} must have {ndim} dimensions")
+
+
+def status_string(status):
+    return lib.lg_status_string(int(status)).decode()
+
+
+def version():
+    return lib.lg_version()
+
+
+def launch_count():
+    """Kernels launched by the library so far in this process."""
+    return int(lib.lg_launch_count())
+
+
+def set_wait_limit_ns(limit_ns):
+    """Bound on each wait inside lora_linear's pipeline; 0 restores the default."""
+    lib.lg_set_wait_limit_ns(int(limit_ns))
+
+
+def get_last_device_error(device=None):
+    """Synchronize the current stream and read/clear the device error word (a status code)."""
+    device = torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)
+    with torch.cuda.device(device):
+        return lib.lg_get_last_device_error(_stream(device))
+
+
+def lora_merge(As, Bs, scales, A_cat=None, B_cat=None):
+    """A_cat = [s_i A_i] stacked along the rank axis, B_cat = [B_i] side by side (FP32)."""
+    n = len(As)
+    if n != len(Bs) or n != len(scales):
+        raise ValueError("As, Bs and scales must have equal length")
+    for i, (A, B) in enumerate(zip(As, Bs)):
+        _need(A, torch.float32, f"A[{i}]", 2)
+        _need(B, torch.float32, f"B[{i}]", 2)
+    d_in = As[0].shape[1]
+    d_out = Bs[0].shape[0]
+    ranks = [A.shape[0] for A in As]
+    for A, B in zip(As, Bs):
+        if A.shape[1] != d_in or B.shape[0] != d_out or B.shape[1] != A.shape[0]:
+            raise ValueError("adapter factor shapes disagree")
+    R = sum(ranks)
+    dev = As[0].device
+    if A_cat is None:
+        A_cat = torch.empty((R, d_in), dtype=torch.float32, device=dev)
+    if B_cat is None:
+        B_cat = torch.empty((d_out, R), dtype=torch.float32, device=dev)
+    _need(A_cat, torch.float32, "A_cat", 2)
+    _need(B_cat, torch.float32, "B_cat", 2)
+    a_ptrs = (ctypes.c_void_p * n)(*[A.data_ptr() for A in As])
+    b_ptrs = (ctypes.c_void_p * n)(*[B.data_ptr() for B in Bs])
+    r_arr = (ctypes.c_int * n)(*ranks)
+    s_arr = (ctypes.c_float * n)(*[float(s) for s in scales])
+    with torch.cuda.device(dev):
+        st = lib.lg_lora_merge(n, a_ptrs, b_ptrs, r_arr, s_arr, d_in, d_out, _ptr(A_cat), _ptr(B_cat), _stream(dev))
+    _check(st, "lg_lora_merge")
+    return A_cat, B_cat
+
+
+def lora_linear_workspace_size(M, K, N, R):
+    return int(lib.lg_lora_linear_workspace_size(int(M), int(K), int(N), int(R)))
+
+
+def lora_linear(x, W, A_cat, B_cat, y=None, workspace=None):
+    """y = x W^T + (x A_cat^T) B_cat^T; bf16 x [M, K], W [N, K]; FP32 A_cat [R, K], B_cat [N, R]."""
+    _need(x, torch.bfloat16, "x", 2)
+    _need(W, torch.bfloat16, "W", 2)
+    M, K = x.shape
+    N = W.shape[0]
+    if W.shape[1] != K:
+        raise ValueError("W must be [N, K]")
+    R = 0
+    if A_cat is not None and A_cat.numel() > 0:
+        _need(A_cat, torch.float32, "A_cat", 2)
+        _need(B_cat, torch.float32, "B_cat", 2)
+        R = A_cat.shape[0]
+        if A_cat.shape[1] != K or tuple(B_cat.shape) != (N, R):
+            raise ValueError("A_cat must be [R, K] and B_cat [N, R]")
+    else:
+        A_cat = B_cat = None
+    if y is None:
+        y = torch.empty((M, N), dtype=torch.bfloat16, device=x.device)
+    _need(y, torch.bfloat16, "y", 2)
+    need = lora_linear_workspace_size(M, K, N, R)
+    if workspace is None and need > 0:
+        workspace = torch.empty(need, dtype=torch.uint8, device=x.device)
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    with torch.cuda.device(x.device):
+        st = lib.lg_lora_linear(_ptr(x), _ptr(W), _ptr(A_cat), _ptr(B_cat), _ptr(y), M, K, N, R,
+                                _ptr(workspace), ws_bytes, _stream(x.device))
+    _check(st, "lg_lora_linear")
+    return y
+
+
+def renoise(up, sigma, seed, offset=0, out=None):
+    """x = (1 - sigma) up + sigma eps(seed, offset + i); FP32."""
+    _need(up, torch.float32, "up")
+    if out is None:
+        out = torch.empty_like(up)
+    _need(out, torch.float32, "out")
+    if out.numel() != up.numel():
+        raise ValueError("out must have as many elements as up")
+    with torch.cuda.device(up.device):
+        st = lib.lg_renoise(_ptr(up), _ptr(out), up.numel(), float(sigma), int(seed), int(offset), _stream(up.device))
+    _check(st, "lg_renoise")
+    return out
+
+
+def euler_step(x, v, sigma, sigma_next):
+    """In place: x += (sigma_next - sigma) v; FP32."""
+    _need(x, torch.float32, "x")
+    _need(v, torch.float32, "v")
+    if x.numel() != v.numel():
+        raise ValueError("x and v must have the same number of elements")
+    with torch.cuda.device(x.device):
+        st = lib.lg_euler_step(_ptr(x), _ptr(v), x.numel(), float(sigma), float(sigma_next), _stream(x.device))
+    _check(st, "lg_euler_step")
+    return x
+
+
+def philox_u32(n_blocks, seed, block_offset=0, out=None, device=None):
+    """Raw Philox4x32-10 words, 4 per block, as an int32 tensor holding the uint32 bits."""
+    if out is None:
+        device = torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)
+        out = torch.empty(4 * int(n_blocks), dtype=torch.int32, device=device)
+    _need(out, torch.int32, "out")
+    if out.numel() < 4 * n_blocks:
+        raise ValueError("out too small")
+    with torch.cuda.device(out.device):
+        st = lib.lg_philox_u32(_ptr(out), int(n_blocks), int(seed), int(block_offset), _stream(out.device))
+    _check(st, "lg_philox_u32")
+    return out
+
+
+def philox_normal(n, seed, offset=0, out=None, device=None):
+    """eps[i] = element offset + i of the Box-Muller normal stream (FP32)."""
+    if out is None:
+        device = torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)
+        out = torch.empty(int(n), dtype=torch.float32, device=device)
+    _need(out, torch.float32, "out")
+    if out.numel() < n:
+        raise ValueError("out too small")
+    with torch.cuda.device(out.device):
+        st = lib.lg_philox_normal(_ptr(out), int(n), int(seed), int(offset), _stream(out.device))
+    _check(st, "lg_philox_normal")
+    return out

@@ -1,0 +1,259 @@
+// C ABI entry points (include/lora_gemm.h): argument validation, device
+// checks and kernel launches.  Nothing here allocates device memory.
+#include <atomic>
+#include <cmath>
+#include <mutex>
+
+#include "../../include/lora_gemm.h"
+#include "lg_internal.h"
+
+namespace {
+
+constexpr uint64_t kDefaultWaitLimitNs = 4000000000ull;
+constexpr int kMaxRank = 576;
+constexpr int kMaxDim = 1 << 20;
+
+std::atomic<uint64_t> g_launches{0};
+std::atomic<uint64_t> g_wait_limit_ns{kDefaultWaitLimitNs};
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// [a, a + na) and [b, b + nb) in bytes.
+bool overlaps(const void* a, uint64_t na, const void* b, uint64_t nb) {
+  const uintptr_t pa = reinterpret_cast<uintptr_t>(a), pb = reinterpret_cast<uintptr_t>(b);
+  return pa < pb + nb && pb < pa + na;
+}
+
+uint64_t align256(uint64_t v) { return (v + 255u) & ~(uint64_t)255u; }
+
+struct DeviceInfo {
+  bool known = false;
+  bool sm100 = false;
+  int sm_count = 0;
+};
+
+// Compute capability and SM count of the current device (cached).
+lg_status current_device(int* sm_count) {
+  static std::mutex mu;
+  static DeviceInfo cache[64];
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess) {
+    cudaGetLastError();
+    return LG_ERR_CUDA;
+  }
+  std::lock_guard<std::mutex> lock(mu);
+  DeviceInfo local;
+  DeviceInfo* info = (dev >= 0 && dev < 64) ? &cache[dev] : &local;
+  if (!info->known) {
+    int major = 0, minor = 0, sms = 0;
+    if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) {
+      cudaGetLastError();
+      return LG_ERR_CUDA;
+    }
+    info->sm100 = (major == 10 && minor == 0);
+    info->sm_count = sms;
+    info->known = true;
+  }
+  if (!info->sm100) return LG_ERR_NOT_SM100;
+  *sm_count = info->sm_count;
+  return LG_OK;
+}
+
+lg_status launched(cudaError_t e, uint64_t kernels) {
+  if (e != cudaSuccess) return LG_ERR_CUDA;
+  g_launches.fetch_add(kernels, std::memory_order_relaxed);
+  return LG_OK;
+}
+
+cudaStream_t as_stream(void* s) { return reinterpret_cast<cudaStream_t>(s); }
+
+}  // namespace
+
+extern "C" {
+
+const char* lg_status_string(int status) {
+  switch (status) {
+    case LG_OK: return "ok";
+    case LG_ERR_INVALID_ARG: return "invalid argument";
+    case LG_ERR_UNSUPPORTED_SHAPE: return "unsupported shape";
+    case LG_ERR_MISALIGNED: return "pointer not 16-byte aligned";
+    case LG_ERR_WORKSPACE: return "workspace missing or too small";
+    case LG_ERR_CUDA: return "CUDA call failed";
+    case LG_ERR_DEVICE_TIMEOUT: return "bounded wait inside a kernel ran out";
+    case LG_ERR_NOT_SM100: return "current device is not compute capability 10.0 (sm_100a)";
+    default: return "unknown status";
+  }
+}
+
+int lg_version(void) { return 10000; }
+
+uint64_t lg_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
+
+void lg_set_wait_limit_ns(uint64_t limit_ns) {
+  g_wait_limit_ns.store(limit_ns == 0 ? kDefaultWaitLimitNs : limit_ns, std::memory_order_relaxed);
+}
+
+lg_status lg_get_last_device_error(void* stream) {
+  int v = 0;
+  if (lg::read_and_clear_device_error(as_stream(stream), &v) != cudaSuccess) {
+    cudaGetLastError();
+    return LG_ERR_CUDA;
+  }
+  return (lg_status)v;
+}
+
+lg_status lg_lora_merge(int n_adapters, const float* const* A, const float* const* B, const int* ranks,
+                        const float* scales, int d_in, int d_out, float* A_cat, float* B_cat, void* stream) {
+  if (n_adapters < 1 || n_adapters > lg::kMaxAdapters || !A || !B || !ranks || !scales || !A_cat || !B_cat)
+    return LG_ERR_INVALID_ARG;
+  if (d_in < 1 || d_out < 1 || d_in > kMaxDim || d_out > kMaxDim || d_in % 4 || d_out % 4)
+    return LG_ERR_UNSUPPORTED_SHAPE;
+  lg::MergeAParams pa{};
+  lg::MergeBParams pb{};
+  int R = 0;
+  for (int i = 0; i < n_adapters; ++i) {
+    if (!A[i] || !B[i] || !std::isfinite(scales[i])) return LG_ERR_INVALID_ARG;
+    if (ranks[i] < 1 || ranks[i] % 4 || ranks[i] > kMaxDim) return LG_ERR_UNSUPPORTED_SHAPE;
+    if (!aligned16(A[i]) || !aligned16(B[i])) return LG_ERR_MISALIGNED;
+    pa.A[i] = A[i];
+    pa.scale[i] = scales[i];
+    pa.row_off[i] = R;
+    pb.B[i] = B[i];
+    pb.col_off[i] = R;
+    R += ranks[i];
+    if (R > kMaxDim) return LG_ERR_UNSUPPORTED_SHAPE;
+  }
+  pa.row_off[n_adapters] = R;
+  pb.col_off[n_adapters] = R;
+  pa.n_adapters = pb.n_adapters = n_adapters;
+  pa.d_in = d_in;
+  pb.d_out = d_out;
+  if (!aligned16(A_cat) || !aligned16(B_cat)) return LG_ERR_MISALIGNED;
+  const uint64_t bytesA = 4ull * R * d_in, bytesB = 4ull * R * d_out;
+  if (overlaps(A_cat, bytesA, B_cat, bytesB)) return LG_ERR_INVALID_ARG;
+  for (int i = 0; i < n_adapters; ++i) {
+    const uint64_t ai = 4ull * ranks[i] * d_in, bi = 4ull * ranks[i] * d_out;
+    if (overlaps(A_cat, bytesA, A[i], ai) || overlaps(A_cat, bytesA, B[i], bi) ||
+        overlaps(B_cat, bytesB, A[i], ai) || overlaps(B_cat, bytesB, B[i], bi))
+      return LG_ERR_INVALID_ARG;
+  }
+  int sms = 0;
+  lg_status st = current_device(&sms);
+  if (st != LG_OK) return st;
+  return launched(lg::launch_merge(pa, pb, A_cat, B_cat, sms, as_stream(stream)), 2);
+}
+
+size_t lg_lora_linear_workspace_size(int64_t M, int K, int N, int R) {
+  if (M < 0 || K < 64 || N < 32 || K % 64 || N % 32 || K > kMaxDim || N > kMaxDim) return 0;
+  if (R < 0 || R % 64 || R > kMaxRank) return 0;
+  if (R == 0) return 0;
+  return (size_t)(align256(2ull * R * K) + align256(2ull * N * R));
+}
+
+lg_status lg_lora_linear(const void* x, const void* W, const float* A_cat, const float* B_cat, void* y, int64_t M,
+                         int K, int N, int R, void* workspace, size_t ws_bytes, void* stream) {
+  if (M < 0 || K < 0 || N < 0 || R < 0) return LG_ERR_INVALID_ARG;
+  if (M >= (int64_t)1 << 31 || K < 64 || N < 32 || K % 64 || N % 32 || K > kMaxDim || N > kMaxDim)
+    return LG_ERR_UNSUPPORTED_SHAPE;
+  if (R % 64 || R > kMaxRank) return LG_ERR_UNSUPPORTED_SHAPE;
+  if (!x || !W || !y) return LG_ERR_INVALID_ARG;
+  if (R > 0 && (!A_cat || !B_cat)) return LG_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(W) || !aligned16(y)) return LG_ERR_MISALIGNED;
+  if (R > 0 && (!aligned16(A_cat) || !aligned16(B_cat))) return LG_ERR_MISALIGNED;
+  const size_t need = lg_lora_linear_workspace_size(M, K, N, R);
+  if (R > 0) {
+    if (!workspace || ws_bytes < need) return LG_ERR_WORKSPACE;
+    if (!aligned16(workspace)) return LG_ERR_MISALIGNED;
+  }
+  const uint64_t bx = 2ull * M * K, bw = 2ull * N * K, by = 2ull * M * N;
+  if (M > 0) {
+    if (overlaps(y, by, x, bx) || overlaps(y, by, W, bw)) return LG_ERR_INVALID_ARG;
+    if (R > 0 && (overlaps(y, by, A_cat, 4ull * R * K) || overlaps(y, by, B_cat, 4ull * N * R) ||
+                  overlaps(y, by, workspace, need)))
+      return LG_ERR_INVALID_ARG;
+  }
+  if (R > 0 && (overlaps(workspace, need, A_cat, 4ull * R * K) || overlaps(workspace, need, B_cat, 4ull * N * R) ||
+                overlaps(workspace, need, x, bx) || overlaps(workspace, need, W, bw)))
+    return LG_ERR_INVALID_ARG;
+  if (M == 0) return LG_OK;
+  int sms = 0;
+  lg_status st = current_device(&sms);
+  if (st != LG_OK) return st;
+  cudaStream_t s = as_stream(stream);
+  uint16_t* wsA = nullptr;
+  uint16_t* wsB = nullptr;
+  if (R > 0) {
+    wsA = reinterpret_cast<uint16_t*>(workspace);
+    wsB = reinterpret_cast<uint16_t*>(reinterpret_cast<uint8_t*>(workspace) + align256(2ull * R * K));
+    st = launched(lg::launch_prep_bf16(A_cat, B_cat, wsA, wsB, (int64_t)R * K, (int64_t)N * R, sms, s), 1);
+    if (st != LG_OK) return st;
+  }
+  lg::LinearLaunch p;
+  p.x = x;
+  p.W = W;
+  p.A_bf16 = wsA;
+  p.B_bf16 = wsB;
+  p.y = y;
+  p.M = M;
+  p.K = K;
+  p.N = N;
+  p.R = R;
+  p.sm_count = sms;
+  p.wait_limit_ns = g_wait_limit_ns.load(std::memory_order_relaxed);
+  bool driver_failed = false;
+  cudaError_t e = lg::launch_lora_linear(p, s, &driver_failed);
+  if (e != cudaSuccess) cudaGetLastError();
+  return launched(e, 1);
+}
+
+lg_status lg_renoise(const float* up, float* x, int64_t n, float sigma, uint64_t seed, uint64_t offset,
+                     void* stream) {
+  if (n < 0 || !std::isfinite(sigma) || sigma < 0.0f || sigma > 1.0f || offset % 4) return LG_ERR_INVALID_ARG;
+  if (n == 0) return LG_OK;
+  if (!up || !x) return LG_ERR_INVALID_ARG;
+  if (!aligned16(up) || !aligned16(x)) return LG_ERR_MISALIGNED;
+  if (up != x && overlaps(up, 4ull * n, x, 4ull * n)) return LG_ERR_INVALID_ARG;
+  int sms = 0;
+  lg_status st = current_device(&sms);
+  if (st != LG_OK) return st;
+  return launched(lg::launch_renoise(up, x, n, sigma, seed, offset, sms, as_stream(stream)), 1);
+}
+
+lg_status lg_euler_step(float* x, const float* v, int64_t n, float sigma, float sigma_next, void* stream) {
+  if (n < 0 || !std::isfinite(sigma) || !std::isfinite(sigma_next)) return LG_ERR_INVALID_ARG;
+  if (n == 0) return LG_OK;
+  if (!x || !v) return LG_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(v)) return LG_ERR_MISALIGNED;
+  if (overlaps(x, 4ull * n, v, 4ull * n)) return LG_ERR_INVALID_ARG;
+  int sms = 0;
+  lg_status st = current_device(&sms);
+  if (st != LG_OK) return st;
+  const float dt = sigma_next - sigma;
+  return launched(lg::launch_euler(x, v, n, dt, sms, as_stream(stream)), 1);
+}
+
+lg_status lg_philox_u32(uint32_t* out, int64_t n_blocks, uint64_t seed, uint64_t block_offset, void* stream) {
+  if (n_blocks < 0) return LG_ERR_INVALID_ARG;
+  if (n_blocks == 0) return LG_OK;
+  if (!out) return LG_ERR_INVALID_ARG;
+  if (!aligned16(out)) return LG_ERR_MISALIGNED;
+  int sms = 0;
+  lg_status st = current_device(&sms);
+  if (st != LG_OK) return st;
+  return launched(lg::launch_philox_u32(out, n_blocks, seed, block_offset, sms, as_stream(stream)), 1);
+}
+
+lg_status lg_philox_normal(float* eps, int64_t n, uint64_t seed, uint64_t offset, void* stream) {
+  if (n < 0 || offset % 4) return LG_ERR_INVALID_ARG;
+  if (n == 0) return LG_OK;
+  if (!eps) return LG_ERR_INVALID_ARG;
+  if (!aligned16(eps)) return LG_ERR_MISALIGNED;
+  int sms = 0;
+  lg_status st = current_device(&sms);
+  if (st != LG_OK) return st;
+  return launched(lg::launch_philox_normal(eps, n, seed, offset, sms, as_stream(stream)), 1);
+}
+
+}  // extern "C"

@@ -1,0 +1,219 @@
+// HBM-bound kernels of the refiner hot path: Philox stream, Gaussian noise,
+// partial re-noise, the Euler update, the rank-axis LoRA merge and the bf16
+// copies of the merged factors.  All are grid-stride loops over 16-byte
+// vectors (one float4 = one Philox block of 4 elements), sized to a few waves
+// of the SMs, with a scalar tail.
+//
+// Re-noise and Euler follow "Open-H3-Regenerate-2K: High-Resolution Video
+// Refinement with Few-Step Diffusion", section "Three steps instead of
+// dozens"; the merge follows "Open-H3-Regenerate-2K：MiniMax H3 的开源 4K
+// 精修方案", section "三个步如何完成工作".
+#include <algorithm>
+
+#include "lg_device.cuh"
+#include "lg_internal.h"
+
+namespace lg {
+
+namespace {
+
+constexpr int kThreads = 256;
+
+__device__ __forceinline__ int64_t gtid() { return (int64_t)blockIdx.x * blockDim.x + threadIdx.x; }
+__device__ __forceinline__ int64_t gstride() { return (int64_t)gridDim.x * blockDim.x; }
+
+__global__ void __launch_bounds__(kThreads) k_philox_u32(uint4* __restrict__ out, int64_t n_blocks, uint32_t k0,
+                                                         uint32_t k1, uint64_t block0) {
+  for (int64_t b = gtid(); b < n_blocks; b += gstride()) {
+    const Words4 r = philox4x32_10(block0 + (uint64_t)b, k0, k1);
+    out[b] = make_uint4(r.w0, r.w1, r.w2, r.w3);
+  }
+}
+
+// The four normals of Philox block `block`.
+__device__ __forceinline__ void normals4(uint64_t block, uint32_t k0, uint32_t k1, double (&e)[4]) {
+  const Words4 r = philox4x32_10(block, k0, k1);
+  box_muller(r.w0, r.w1, e[0], e[1]);
+  box_muller(r.w2, r.w3, e[2], e[3]);
+}
+
+__global__ void __launch_bounds__(kThreads) k_philox_normal(float* __restrict__ eps, int64_t n, uint32_t k0,
+                                                            uint32_t k1, uint64_t block0) {
+  const int64_t n_blocks = (n + 3) / 4;
+  for (int64_t b = gtid(); b < n_blocks; b += gstride()) {
+    double e[4];
+    normals4(block0 + (uint64_t)b, k0, k1, e);
+    if (4 * b + 4 <= n) {
+      reinterpret_cast<float4*>(eps)[b] = make_float4((float)e[0], (float)e[1], (float)e[2], (float)e[3]);
+    } else {
+      for (int t = 0; t < 4 && 4 * b + t < n; ++t) eps[4 * b + t] = (float)e[t];
+    }
+  }
+}
+
+// x = (1 - sigma) up + sigma eps, blended in double from the unrounded eps
+// and rounded once to FP32.  x may alias up (each element is read before it
+// is written by the same thread), so neither pointer is restrict.
+__global__ void __launch_bounds__(kThreads) k_renoise(const float* up, float* x, int64_t n,
+                                                      double sigma, uint32_t k0, uint32_t k1, uint64_t block0) {
+  const double keep = 1.0 - sigma;
+  const int64_t n_blocks = (n + 3) / 4;
+  for (int64_t b = gtid(); b < n_blocks; b += gstride()) {
+    double e[4];
+    normals4(block0 + (uint64_t)b, k0, k1, e);
+    if (4 * b + 4 <= n) {
+      const float4 u = __ldcs(reinterpret_cast<const float4*>(up) + b);
+      float4 o;
+      o.x = (float)fma(sigma, e[0], keep * (double)u.x);
+      o.y = (float)fma(sigma, e[1], keep * (double)u.y);
+      o.z = (float)fma(sigma, e[2], keep * (double)u.z);
+      o.w = (float)fma(sigma, e[3], keep * (double)u.w);
+      __stcs(reinterpret_cast<float4*>(x) + b, o);
+    } else {
+      for (int t = 0; t < 4 && 4 * b + t < n; ++t) {
+        x[4 * b + t] = (float)fma(sigma, e[t], keep * (double)up[4 * b + t]);
+      }
+    }
+  }
+}
+
+// x += dt v with dt = sigma_next - sigma taken in FP32 (exact for the
+// schedule by Sterbenz's lemma); one fused multiply-add per element.
+constexpr int kEulerUnroll = 4;
+__global__ void __launch_bounds__(kThreads) k_euler(float* __restrict__ x, const float* __restrict__ v, int64_t n,
+                                                    float dt) {
+  const int64_t n4 = n / 4;
+  float4* x4 = reinterpret_cast<float4*>(x);
+  const float4* v4 = reinterpret_cast<const float4*>(v);
+  const int64_t stride = gstride();
+  int64_t i = gtid();
+  for (; i + (kEulerUnroll - 1) * stride < n4; i += kEulerUnroll * stride) {
+    float4 a[kEulerUnroll], b[kEulerUnroll];
+#pragma unroll
+    for (int u = 0; u < kEulerUnroll; ++u) {
+      a[u] = x4[i + u * stride];
+      b[u] = __ldcs(v4 + i + u * stride);
+    }
+#pragma unroll
+    for (int u = 0; u < kEulerUnroll; ++u) {
+      a[u].x = fmaf(dt, b[u].x, a[u].x);
+      a[u].y = fmaf(dt, b[u].y, a[u].y);
+      a[u].z = fmaf(dt, b[u].z, a[u].z);
+      a[u].w = fmaf(dt, b[u].w, a[u].w);
+      x4[i + u * stride] = a[u];
+    }
+  }
+  for (; i < n4; i += stride) {
+    float4 a = x4[i];
+    const float4 b = __ldcs(v4 + i);
+    a.x = fmaf(dt, b.x, a.x);
+    a.y = fmaf(dt, b.y, a.y);
+    a.z = fmaf(dt, b.z, a.z);
+    a.w = fmaf(dt, b.w, a.w);
+    x4[i] = a;
+  }
+  if (gtid() == 0) {
+    for (int64_t t = 4 * n4; t < n; ++t) x[t] = fmaf(dt, v[t], x[t]);
+  }
+}
+
+// A_cat[off_i + r][k] = s_i A_i[r][k]  (float4 granularity; d_in % 4 == 0).
+__global__ void __launch_bounds__(kThreads) k_merge_a(const MergeAParams p, float* __restrict__ A_cat) {
+  const int64_t q = p.d_in / 4;
+  const int64_t total = (int64_t)p.row_off[p.n_adapters] * q;
+  for (int64_t i = gtid(); i < total; i += gstride()) {
+    const int row = (int)(i / q);
+    const int64_t c = i - (int64_t)row * q;
+    int a = 0;
+    while (a + 1 < p.n_adapters && row >= p.row_off[a + 1]) ++a;
+    const float s = p.scale[a];
+    const float4 v = reinterpret_cast<const float4*>(p.A[a])[(int64_t)(row - p.row_off[a]) * q + c];
+    reinterpret_cast<float4*>(A_cat)[i] = make_float4(s * v.x, s * v.y, s * v.z, s * v.w);
+  }
+}
+
+// B_cat[o][off_i + r] = B_i[o][r]  (ranks % 4 == 0, so a float4 never
+// straddles two adapters).
+__global__ void __launch_bounds__(kThreads) k_merge_b(const MergeBParams p, float* __restrict__ B_cat) {
+  const int R = p.col_off[p.n_adapters];
+  const int q = R / 4;
+  const int64_t total = (int64_t)p.d_out * q;
+  for (int64_t i = gtid(); i < total; i += gstride()) {
+    const int64_t o = i / q;
+    const int col = (int)(i - o * q) * 4;
+    int a = 0;
+    while (a + 1 < p.n_adapters && col >= p.col_off[a + 1]) ++a;
+    const int r_a = p.col_off[a + 1] - p.col_off[a];
+    const float4 v = *reinterpret_cast<const float4*>(p.B[a] + o * r_a + (col - p.col_off[a]));
+    reinterpret_cast<float4*>(B_cat)[i] = v;
+  }
+}
+
+// FP32 -> bf16 round-to-nearest-even, two arrays in one launch (n % 4 == 0).
+__global__ void __launch_bounds__(kThreads) k_prep_bf16(const float* __restrict__ a, const float* __restrict__ b,
+                                                        uint16_t* __restrict__ da, uint16_t* __restrict__ db,
+                                                        int64_t na4, int64_t nb4) {
+  for (int64_t i = gtid(); i < na4 + nb4; i += gstride()) {
+    const bool first = i < na4;
+    const int64_t j = first ? i : i - na4;
+    const float4 v = reinterpret_cast<const float4*>(first ? a : b)[j];
+    uint2 o;
+    o.x = pack_bf16x2(v.x, v.y);
+    o.y = pack_bf16x2(v.z, v.w);
+    reinterpret_cast<uint2*>(first ? da : db)[j] = o;
+  }
+}
+
+}  // namespace
+
+int elementwise_grid(int64_t work, int sm_count) {
+  const int64_t want = (work + kThreads - 1) / kThreads;
+  const int64_t cap = (int64_t)std::max(sm_count, 1) * 8;  // 8 x 256 threads = 2048 per SM
+  return (int)std::max<int64_t>(1, std::min(want, cap));
+}
+
+cudaError_t launch_philox_u32(uint32_t* out, int64_t n_blocks, uint64_t seed, uint64_t block_offset, int sm_count,
+                              cudaStream_t s) {
+  k_philox_u32<<<elementwise_grid(n_blocks, sm_count), kThreads, 0, s>>>(
+      reinterpret_cast<uint4*>(out), n_blocks, (uint32_t)seed, (uint32_t)(seed >> 32), block_offset);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_philox_normal(float* eps, int64_t n, uint64_t seed, uint64_t offset, int sm_count,
+                                 cudaStream_t s) {
+  k_philox_normal<<<elementwise_grid((n + 3) / 4, sm_count), kThreads, 0, s>>>(eps, n, (uint32_t)seed,
+                                                                               (uint32_t)(seed >> 32), offset / 4);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_renoise(const float* up, float* x, int64_t n, float sigma, uint64_t seed, uint64_t offset,
+                           int sm_count, cudaStream_t s) {
+  k_renoise<<<elementwise_grid((n + 3) / 4, sm_count), kThreads, 0, s>>>(up, x, n, (double)sigma, (uint32_t)seed,
+                                                                         (uint32_t)(seed >> 32), offset / 4);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_euler(float* x, const float* v, int64_t n, float dt, int sm_count, cudaStream_t s) {
+  k_euler<<<elementwise_grid(std::max<int64_t>(n / 4, 1), sm_count), kThreads, 0, s>>>(x, v, n, dt);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_merge(const MergeAParams& pa, const MergeBParams& pb, float* A_cat, float* B_cat, int sm_count,
+                         cudaStream_t s) {
+  const int64_t wa = (int64_t)pa.row_off[pa.n_adapters] * (pa.d_in / 4);
+  const int64_t wb = (int64_t)pb.d_out * (pb.col_off[pb.n_adapters] / 4);
+  k_merge_a<<<elementwise_grid(wa, sm_count), kThreads, 0, s>>>(pa, A_cat);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  k_merge_b<<<elementwise_grid(wb, sm_count), kThreads, 0, s>>>(pb, B_cat);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_prep_bf16(const float* A_cat, const float* B_cat, uint16_t* dstA, uint16_t* dstB, int64_t nA,
+                             int64_t nB, int sm_count, cudaStream_t s) {
+  const int64_t w = nA / 4 + nB / 4;
+  k_prep_bf16<<<elementwise_grid(w, sm_count), kThreads, 0, s>>>(A_cat, B_cat, dstA, dstB, nA / 4, nB / 4);
+  return cudaGetLastError();
+}
+
+}  // namespace lg

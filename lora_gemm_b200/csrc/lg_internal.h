@@ -1,0 +1,63 @@
+// Internal host-side interface between the C ABI layer (lg_api.cu) and the
+// kernel translation units.  Not part of the public ABI.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+namespace lg {
+
+constexpr int kMaxAdapters = 8;
+
+struct MergeAParams {
+  const float* A[kMaxAdapters];
+  float scale[kMaxAdapters];
+  int row_off[kMaxAdapters + 1];  // prefix sums of the ranks
+  int n_adapters;
+  int d_in;
+};
+
+struct MergeBParams {
+  const float* B[kMaxAdapters];
+  int col_off[kMaxAdapters + 1];
+  int n_adapters;
+  int d_out;
+};
+
+// Grid size for a grid-stride elementwise kernel over `work` items.
+int elementwise_grid(int64_t work, int sm_count);
+
+cudaError_t launch_philox_u32(uint32_t* out, int64_t n_blocks, uint64_t seed, uint64_t block_offset, int sm_count,
+                              cudaStream_t s);
+cudaError_t launch_philox_normal(float* eps, int64_t n, uint64_t seed, uint64_t offset, int sm_count,
+                                 cudaStream_t s);
+cudaError_t launch_renoise(const float* up, float* x, int64_t n, float sigma, uint64_t seed, uint64_t offset,
+                           int sm_count, cudaStream_t s);
+cudaError_t launch_euler(float* x, const float* v, int64_t n, float dt, int sm_count, cudaStream_t s);
+cudaError_t launch_merge(const MergeAParams& pa, const MergeBParams& pb, float* A_cat, float* B_cat, int sm_count,
+                         cudaStream_t s);
+// FP32 -> bf16 (RNE) of A_cat [R, K] and B_cat [N, R] into dstA / dstB.
+cudaError_t launch_prep_bf16(const float* A_cat, const float* B_cat, uint16_t* dstA, uint16_t* dstB,
+                             int64_t nA, int64_t nB, int sm_count, cudaStream_t s);
+
+// Merged-LoRA linear (tcgen05 kernel).  Factors already in bf16.
+struct LinearLaunch {
+  const void* x;
+  const void* W;
+  const uint16_t* A_bf16;  // [R, K]
+  const uint16_t* B_bf16;  // [N, R]
+  void* y;
+  int64_t M;
+  int K, N, R;
+  int sm_count;
+  uint64_t wait_limit_ns;
+};
+// Returns cudaSuccess or the failing CUDA error; *driver_failed is set when
+// the tensor-map encoder (driver API) is missing or rejects a map.
+cudaError_t launch_lora_linear(const LinearLaunch& p, cudaStream_t s, bool* driver_failed);
+
+// Device error word of the current device: read and clear (synchronous on s).
+cudaError_t read_and_clear_device_error(cudaStream_t s, int* value);
+
+}  // namespace lg

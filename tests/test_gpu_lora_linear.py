@@ -1,0 +1,142 @@
+"""GPU parity of lora_linear (tcgen05 kernel) against the FP64 oracle.
+
+Bar: relative Frobenius error <= 1e-2 against y = x W^T + (x A_cat^T) B_cat^T
+evaluated in FP64 from the exact input values.  The kernel rounds the merged
+factors and h = x A_cat^T to bf16 and y to bf16 (each ~2^-9 relative), so the
+expected error is a few 1e-3.  Small shapes compare every element and cover
+ragged M and N tails, rank 0 / 64 / 576 and a single K block; the full-size
+workloads compare 512 seeded sample rows, with the factors merged by the
+oracle from the same adapters.
+"""
+
+import numpy as np
+import pytest
+import torch
+
+import lora_gemm_b200 as lg
+from lora_gemm_b200 import synth
+from oracle import lora as olora
+from tests.util import rel_fro
+
+pytestmark = pytest.mark.gpu
+DEV = "cuda"
+TOL = 1e-2
+
+
+def _np64(t):
+    return t.detach().float().cpu().numpy().astype(np.float64)
+
+
+def _rand_layer(M, K, N, R, seed, zero_w=False):
+    g = torch.Generator().manual_seed(seed)
+    x = torch.randn(M, K, generator=g).to(torch.bfloat16)
+    W = (torch.randn(N, K, generator=g) * K ** -0.5).to(torch.bfloat16)
+    if zero_w:
+        W.zero_()
+    A = torch.randn(R, K, generator=g) * K ** -0.5
+    B = torch.randn(N, R, generator=g) * 0.1
+    return x.to(DEV), W.to(DEV), A.to(DEV), B.to(DEV)
+
+
+def _check(x, W, A, B, y):
+    ref = olora.lora_linear(_np64(x), _np64(W), _np64(A), _np64(B))
+    err = rel_fro(_np64(y), ref)
+    assert lg.get_last_device_error() == lg.LG_OK
+    return err
+
+
+@pytest.mark.parametrize(
+    "M,K,N,R",
+    [
+        (128, 64, 224, 0),     # one tile, one K block, no LoRA
+        (1, 64, 64, 64),       # single token, N tail inside one tile
+        (127, 128, 192, 64),   # M tail
+        (300, 256, 448, 128),  # three panels, two full tiles
+        (517, 320, 320, 576),  # ragged everything, full rank
+        (2304, 1024, 1024, 576),
+    ],
+)
+def test_small_shapes_full_matrix(M, K, N, R):
+    x, W, A, B = _rand_layer(M, K, N, R, seed=M * 7 + N)
+    y = lg.lora_linear(x, W, A if R else None, B if R else None)
+    err = _check(x, W, A, B, y)
+    assert err <= TOL, err
+
+
+@pytest.mark.parametrize("R", [64, 576])
+def test_lora_path_alone(R):
+    """W = 0: the output is the up-projection of the on-chip h alone."""
+    x, W, A, B = _rand_layer(384, 512, 448, R, seed=R, zero_w=True)
+    y = lg.lora_linear(x, W, A, B)
+    err = _check(x, W, A, B, y)
+    assert err <= TOL, err
+
+
+def test_base_path_alone_many_panels():
+    """R = 0 with more panels than SMs (persistent loop) is a plain GEMM."""
+    x, W, A, B = _rand_layer(148 * 128 * 2 + 77, 256, 448, 0, seed=3)
+    y = lg.lora_linear(x, W, None, None)
+    err = _check(x, W, A, B, y)
+    assert err <= TOL, err
+
+
+def test_tiny_workload_full_matrix():
+    w = synth.WORKLOADS["tiny"]
+    x = synth.activations(w, 1024, 0, DEV)
+    W = synth.weight(w, 0, DEV)
+    As, Bs = synth.adapters(w, 0, DEV)
+    A_cat, B_cat = lg.lora_merge(As, Bs, synth.ADAPTER_SCALES)
+    y = lg.lora_linear(x, W, A_cat, B_cat)
+    rA, rB = olora.lora_merge([_np64(a) for a in As], [_np64(b) for b in Bs], synth.ADAPTER_SCALES)
+    ref = olora.lora_linear(_np64(x), _np64(W), rA, rB)
+    err = rel_fro(_np64(y), ref)
+    assert lg.get_last_device_error() == lg.LG_OK
+    assert err <= TOL, err
+
+
+def _sampled_rows_case(name, layer, n_rows=512):
+    w = synth.WORKLOADS[name]
+    K, N = w.shapes[layer]
+    x = synth.activations(w, K, layer, DEV)
+    W = synth.weight(w, layer, DEV)
+    As, Bs = synth.adapters(w, layer, DEV)
+    A_cat, B_cat = lg.lora_merge(As, Bs, synth.ADAPTER_SCALES)
+    y = lg.lora_linear(x, W, A_cat, B_cat)
+    assert lg.get_last_device_error() == lg.LG_OK
+    rows = np.sort(np.random.default_rng(w.seed * 10 + layer).choice(w.tokens, n_rows, replace=False))
+    rows = np.unique(np.concatenate([rows, [0, w.tokens - 1]]))
+    idx = torch.as_tensor(rows, device=DEV)
+    y_rows = _np64(y.index_select(0, idx))
+    x_rows = _np64(x.index_select(0, idx))
+    del x, y
+    rA, rB = olora.lora_merge([_np64(a) for a in As], [_np64(b) for b in Bs], synth.ADAPTER_SCALES)
+    ref = olora.lora_linear(x_rows, _np64(W), rA, rB)
+    torch.cuda.empty_cache()
+    return rel_fro(y_rows, ref)
+
+
+@pytest.mark.parametrize(
+    "name,layer",
+    [("768p", 0), ("1080p", 0), ("1080p", 1), ("1080p", 2), ("2k", 0), ("2k", 1), ("2k", 2), ("4k", 0), ("4k", 1),
+     ("4k", 2)],
+)
+def test_full_size_sampled_rows(name, layer):
+    err = _sampled_rows_case(name, layer)
+    assert err <= TOL, err
+
+
+def test_wait_timeout_is_reported_and_context_survives():
+    """A wait limit of 1 ns makes the pipeline's waits run out: the kernel
+    records LG_ERR_DEVICE_TIMEOUT, cleans up and returns; the next call with
+    the default limit is correct."""
+    x, W, A, B = _rand_layer(1024, 1024, 896, 576, seed=9)
+    lg.set_wait_limit_ns(1)
+    try:
+        lg.lora_linear(x, W, A, B)
+        status = lg.get_last_device_error()
+    finally:
+        lg.set_wait_limit_ns(0)
+    assert status == lg.LG_ERR_DEVICE_TIMEOUT
+    y = lg.lora_linear(x, W, A, B)
+    err = _check(x, W, A, B, y)
+    assert err <= TOL, err
