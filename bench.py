@@ -183,19 +183,20 @@ def layer_flops(M, K, N, R):
 class Problem:
     """Device-resident inputs and outputs of one 2K step."""
 
-    def __init__(self, w, dev):
+    def __init__(self, w, dev, tokens=None):
         from lora_gemm_b200 import synth
         import lora_gemm_b200 as lg
 
         self.w = w
-        M = w.tokens
+        M = w.tokens if tokens is None else tokens
+        self.M = M
         R = sum(synth.ADAPTER_RANKS)
         self.R = R
         self.layers = []
         x_by_k = {}
         for i, (K, N) in enumerate(w.shapes):
             if K not in x_by_k:
-                x_by_k[K] = synth.activations(w, K, i, dev)
+                x_by_k[K] = synth.activations(w, K, i, dev, M=M)
             As, Bs = synth.adapters(w, i, dev)
             L = {
                 "K": K, "N": N, "x": x_by_k[K], "W": synth.weight(w, i, dev), "As": As, "Bs": Bs,
@@ -239,7 +240,7 @@ def run_step(P, ev=None):
 def bytes_per_kernel(P):
     w = P.w
     n = w.latent_numel
-    M = w.tokens
+    M = P.M
     merge = sum(4 * P.R * (L["K"] + L["N"]) * 2 for L in P.layers)  # read adapters, write merged
     return {"renoise": 8.0 * n, "euler": 12.0 * n, "lora_merge": merge / len(P.layers),
             "lora_linear_min_bytes": [2.0 * (M * L["K"] + L["N"] * L["K"] + M * L["N"]) + 4.0 * P.R * (L["K"] + L["N"])
@@ -253,7 +254,7 @@ def run_ours(args, rank, world, local):
     peaks = load_peaks()
     dev = torch.device("cuda", torch.cuda.current_device())
     w = synth.WORKLOADS[args.workload]
-    P = Problem(w, dev)
+    P = Problem(w, dev, tokens=args.tokens)
     torch.cuda.synchronize()
 
     for _ in range(args.warmup):
@@ -288,7 +289,7 @@ def run_ours(args, rank, world, local):
     per = {}
     for name, s, e in ev:
         per.setdefault(name, []).append(s.elapsed_time(e))
-    M = w.tokens
+    M = P.M
     value = world * M * args.steps / (elapsed_ms * 1e-3)
 
     # Dominant kernel: lora_linear (tensor-bound).
@@ -343,6 +344,7 @@ def run_ours(args, rank, world, local):
             "workload": w.name,
             "latent": list(w.latent_shape),
             "tokens": M,
+            "tokens_override": args.tokens is not None,
             "d": w.d,
             "layers_k_n": [list(s) for s in w.shapes],
             "rank": P.R,
@@ -376,14 +378,22 @@ def run_ours(args, rank, world, local):
 
 
 def load_traffic():
-    """DRAM bytes per lora_linear launch from the committed ncu summary, if current."""
+    """DRAM bytes per lora_linear launch from the committed ncu summary, or None
+    when the summary is missing or was taken on a different kernel source."""
+    import hashlib
+
     path = os.path.join(ROOT, "profiles", "lora_linear_traffic.json")
+    src = os.path.join(ROOT, "lora_gemm_b200", "csrc", "lg_lora_linear.cu")
     try:
         with open(path) as f:
             t = json.load(f)
-        return t.get("traffic_bytes_per_launch")
+        with open(src, "rb") as f:
+            digest = hashlib.sha256(f.read()).hexdigest()
     except (OSError, ValueError):
         return None
+    if t.get("kernel_source_sha256") != digest:
+        return None
+    return t.get("traffic_bytes_per_launch")
 
 
 def run_e2e(P, args, world):
@@ -427,7 +437,7 @@ def run_e2e(P, args, world):
     torch.cuda.synchronize()
     barrier(world)
     ms = max_over_ranks(s.elapsed_time(e), world)
-    return {"value": round(world * P.w.tokens * steps / (ms * 1e-3), 1), "unit": UNIT,
+    return {"value": round(world * P.M * steps / (ms * 1e-3), 1), "unit": UNIT,
             "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h), "steps": steps,
             "ms_per_step": round(ms / steps, 3)}
 
@@ -555,6 +565,8 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    ap.add_argument("--tokens", type=int, default=None,
+                    help="override the token count of the linear layers (profiling runs only)")
     args = ap.parse_args()
     if args.warmup < 3:
         raise SystemExit("--warmup must be >= 3")
