@@ -142,6 +142,39 @@ lg_status lg_lora_linear(const void* x, const void* W, const float* A_cat, const
                          void* workspace, size_t ws_bytes, void* stream);
 
 /* ------------------------------------------------------------------------
+ * lg_lora_linear_noalloc -- lg_lora_linear for callers that cannot allocate
+ * device memory.  The pages have no counterpart; this is an interface
+ * addition of this library.
+ *
+ * Some callers have no device allocator at the point of the call: a plugin
+ * inside an inference engine whose device memory is planned before the run
+ * and which may not allocate when it is enqueued, or a serving loop that must
+ * never call cudaMalloc (it synchronizes the device and stalls every other
+ * stream).  They cannot provide lg_lora_linear's workspace.  This entry point
+ * takes the same arguments minus the workspace and keeps the bf16 copies of
+ * the merged factors in an array of LG_NOALLOC_SCRATCH_BYTES that is part of
+ * the library's device image: every GPU on which the library's kernels are
+ * loaded holds that memory until the process exits.  The call itself
+ * allocates nothing (no cudaMalloc, cudaFree or allocating library routine).
+ *
+ *   - Result, validation, arithmetic and kernels are those of lg_lora_linear.
+ *   - Limit: lg_lora_linear_workspace_size(M, K, N, R) must not exceed
+ *     LG_NOALLOC_SCRATCH_BYTES (about 2 (K + N) R bytes; with R = 576 this is
+ *     K + N <= 43,690, e.g. the 7168 -> 7168, 7168 -> 21504 and
+ *     28672 -> 7168 layers); a larger shape returns LG_ERR_WORKSPACE and
+ *     launches nothing.
+ *   - The first call on a device looks up the array's device address on that
+ *     device (cudaGetSymbolAddress, with that device current); make that
+ *     first call before any stream capture.
+ *   - Every call uses the same array.  Calls that can overlap on the GPU
+ *     (different streams without ordering between them) race on it; keep
+ *     such calls on one stream or order them with events.
+ * ---------------------------------------------------------------------- */
+#define LG_NOALLOC_SCRATCH_BYTES ((size_t)48 << 20)
+lg_status lg_lora_linear_noalloc(const void* x, const void* W, const float* A_cat, const float* B_cat,
+                                 void* y, int64_t M, int K, int N, int R, void* stream);
+
+/* ------------------------------------------------------------------------
  * lg_renoise -- partial re-noise of an upscaled latent:
  *
  *   x[i] = (1 - sigma) * up[i] + sigma * eps[offset + i],  i in [0, n)

@@ -6,7 +6,7 @@ the caller does not pass them, and hands raw device pointers plus the current
 CUDA stream to liblora_gemm.so.  All arithmetic runs in the library's CUDA
 kernels; there is no CPU path.  Importing this package fails with ImportError
 when the compiled library is missing (build it with
-``python -m lora_gemm_b200.build``).
+``python lora_gemm_b200/build.py``).
 """
 
 import ctypes
@@ -45,6 +45,11 @@ _SIGNATURES = {
         [_c_void_p, _c_void_p, _c_void_p, _c_void_p, _c_void_p, ctypes.c_int64, ctypes.c_int, ctypes.c_int,
          ctypes.c_int, _c_void_p, ctypes.c_size_t, _c_void_p],
     ),
+    "lg_lora_linear_noalloc": (
+        ctypes.c_int,
+        [_c_void_p, _c_void_p, _c_void_p, _c_void_p, _c_void_p, ctypes.c_int64, ctypes.c_int, ctypes.c_int,
+         ctypes.c_int, _c_void_p],
+    ),
     "lg_renoise": (
         ctypes.c_int,
         [_c_void_p, _c_void_p, ctypes.c_int64, ctypes.c_float, ctypes.c_uint64, ctypes.c_uint64, _c_void_p],
@@ -61,7 +66,7 @@ EXPORTED_SYMBOLS = tuple(_SIGNATURES)
 def _load():
     if not os.path.exists(LIB_PATH):
         raise ImportError(
-            f"lora_gemm CUDA library not found at {LIB_PATH}; build it with `python -m lora_gemm_b200.build`"
+            f"lora_gemm CUDA library not found at {LIB_PATH}; build it with `python lora_gemm_b200/build.py`"
         )
     lib = ctypes.CDLL(LIB_PATH)
     for name, (res, args) in _SIGNATURES.items():
@@ -196,6 +201,29 @@ def lora_linear(x, W, A_cat, B_cat, y=None, workspace=None):
         st = lib.lg_lora_linear(_ptr(x), _ptr(W), _ptr(A_cat), _ptr(B_cat), _ptr(y), M, K, N, R,
                                 _ptr(workspace), ws_bytes, _stream(x.device))
     _check(st, "lg_lora_linear")
+    return y
+
+
+def lora_linear_noalloc(x, W, A_cat, B_cat, y):
+    """lora_linear without a workspace, for callers that cannot allocate device
+    memory at call time: the factor copies go to the library's built-in scratch
+    array (see lg_lora_linear_noalloc in include/lora_gemm.h).  y must be given."""
+    _need(x, torch.bfloat16, "x", 2)
+    _need(W, torch.bfloat16, "W", 2)
+    _need(y, torch.bfloat16, "y", 2)
+    M, K = x.shape
+    N = W.shape[0]
+    R = 0
+    if A_cat is not None and A_cat.numel() > 0:
+        _need(A_cat, torch.float32, "A_cat", 2)
+        _need(B_cat, torch.float32, "B_cat", 2)
+        R = A_cat.shape[0]
+    else:
+        A_cat = B_cat = None
+    with torch.cuda.device(x.device):
+        st = lib.lg_lora_linear_noalloc(_ptr(x), _ptr(W), _ptr(A_cat), _ptr(B_cat), _ptr(y), M, K, N, R,
+                                        _stream(x.device))
+    _check(st, "lg_lora_linear_noalloc")
     return y
 
 
