@@ -1,6 +1,9 @@
 """Build the in-tree CUDA library liblora_gemm.so for sm_100a.
 
-Usage: python -m lora_gemm_b200.build [--verbose]
+Usage: python lora_gemm_b200/build.py [--verbose]
+
+(Run it as a file, not as a module of the package: importing the package
+loads the library this script builds.)
 
 Compiles every csrc/*.cu with nvcc (-gencode arch=compute_100a,code=sm_100a,
 -O3, -lineinfo, no fast-math), links them into one shared library next to

@@ -14,8 +14,14 @@ def pytest_configure(config):
 
 @pytest.fixture(scope="session", autouse=True)
 def _built_library():
-    """Compile liblora_gemm.so if it is missing or older than its sources."""
-    from lora_gemm_b200 import build
+    """Compile liblora_gemm.so if it is missing or older than its sources.
 
-    build.build()
+    The build script is loaded by path: importing the package would load the
+    (possibly stale) library first."""
+    import importlib.util
+
+    spec = importlib.util.spec_from_file_location("_lg_build", os.path.join(ROOT, "lora_gemm_b200", "build.py"))
+    mod = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(mod)
+    mod.build()
     yield
