@@ -82,6 +82,22 @@ lg_status lg_get_last_device_error(void* stream);
  * limit makes the waits run out so the timeout path can be exercised. */
 void lg_set_wait_limit_ns(uint64_t limit_ns);
 
+/* Thread-block cluster size of lg_lora_linear: the CTAs (one per SM) that
+ * share one panel of x -- 1, 2, 4 or 8 -- or 0 (the default) to choose
+ * per shape.  Sharing a panel lets the cluster's CTAs split the N tiles while
+ * the panel is read from DRAM once; each computes its slice of the rank-R
+ * intermediate and they exchange the slices through distributed shared
+ * memory.  For the SM-pair variant the size counts both CTAs of each pair
+ * (2, 4 or 8).  Process-wide; for tuning and tests.  Returns
+ * LG_ERR_INVALID_ARG for other values. */
+lg_status lg_set_cluster_size(int g);
+
+/* MMA variant of lg_lora_linear: 1 = single-SM tcgen05.mma (128-row tiles),
+ * 2 = SM-pair tcgen05.mma.cta_group::2 (256-row tiles, each SM loads half of
+ * every B tile), 0 (the default) = chosen per shape.  Process-wide; for
+ * tuning and tests.  Returns LG_ERR_INVALID_ARG for other values. */
+lg_status lg_set_kernel_variant(int v);
+
 /* ------------------------------------------------------------------------
  * lg_lora_merge -- concatenate n_adapters LoRA adapters along the rank axis.
  *

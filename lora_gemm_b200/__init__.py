@@ -34,6 +34,8 @@ _SIGNATURES = {
     "lg_launch_count": (ctypes.c_uint64, []),
     "lg_get_last_device_error": (ctypes.c_int, [_c_void_p]),
     "lg_set_wait_limit_ns": (None, [ctypes.c_uint64]),
+    "lg_set_cluster_size": (ctypes.c_int, [ctypes.c_int]),
+    "lg_set_kernel_variant": (ctypes.c_int, [ctypes.c_int]),
     "lg_lora_merge": (
         ctypes.c_int,
         [ctypes.c_int, ctypes.POINTER(_c_void_p), ctypes.POINTER(_c_void_p), ctypes.POINTER(ctypes.c_int),
@@ -128,6 +130,16 @@ def launch_count():
 def set_wait_limit_ns(limit_ns):
     """Bound on each wait inside lora_linear's pipeline; 0 restores the default."""
     lib.lg_set_wait_limit_ns(int(limit_ns))
+
+
+def set_cluster_size(g):
+    """SMs sharing one token panel in lora_linear (1, 2, 4, 8, 16; 0 = chosen per shape)."""
+    _check(lib.lg_set_cluster_size(int(g)), "lg_set_cluster_size")
+
+
+def set_kernel_variant(v):
+    """lora_linear MMA variant: 1 single-SM, 2 SM pair, 0 chosen per shape."""
+    _check(lib.lg_set_kernel_variant(int(v)), "lg_set_kernel_variant")
 
 
 def get_last_device_error(device=None):

@@ -95,6 +95,18 @@ void lg_set_wait_limit_ns(uint64_t limit_ns) {
   g_wait_limit_ns.store(limit_ns == 0 ? kDefaultWaitLimitNs : limit_ns, std::memory_order_relaxed);
 }
 
+lg_status lg_set_cluster_size(int g) {
+  if (g != 0 && g != 1 && g != 2 && g != 4 && g != 8) return LG_ERR_INVALID_ARG;
+  lg::set_cluster_override(g);
+  return LG_OK;
+}
+
+lg_status lg_set_kernel_variant(int v) {
+  if (v < 0 || v > 2) return LG_ERR_INVALID_ARG;
+  lg::set_variant_override(v);
+  return LG_OK;
+}
+
 lg_status lg_get_last_device_error(void* stream) {
   int v = 0;
   if (lg::read_and_clear_device_error(as_stream(stream), &v) != cudaSuccess) {

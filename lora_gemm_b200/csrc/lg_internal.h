@@ -57,6 +57,11 @@ struct LinearLaunch {
 // the tensor-map encoder (driver API) is missing or rejects a map.
 cudaError_t launch_lora_linear(const LinearLaunch& p, cudaStream_t s, bool* driver_failed);
 
+// CTAs per cluster sharing one panel in lg_lora_linear (0: chosen per shape).
+void set_cluster_override(int g);
+// MMA variant of lg_lora_linear: 1 single-SM, 2 SM pair (0: chosen per shape).
+void set_variant_override(int v);
+
 // Device error word of the current device: read and clear (synchronous on s).
 cudaError_t read_and_clear_device_error(cudaStream_t s, int* value);
 

@@ -9,27 +9,36 @@
 // "三个步如何完成工作", rank 384 + 128 + 64 = 576 on 312 linear layers); the
 // pages give no kernel design, so everything below is this library's.
 //
-// Design (one CTA per SM, persistent over 128-row token panels):
-//   * TMEM (512 columns x 128 lanes, one lane per token row) holds the FP32
-//     accumulator of one 128 x 224 output tile in columns [0, 224) and the
-//     panel's rank-R intermediate h = x A_cat^T as packed bf16 pairs in
-//     columns [224, 224 + R/2) -- 288 columns for R = 576.  h is computed
-//     once per panel and never leaves the SM.
-//   * Phase A (per panel): for each 192-wide rank chunk, a K loop of
-//     tcgen05.mma (A = x tile, B = A_cat tile, both from shared memory)
-//     accumulates the chunk of h in FP32 in the accumulator columns; the
-//     epilogue warps round it to bf16 and store it into the h columns.
-//   * Phase B (per 224-wide N tile): a K loop x W^T into the accumulator,
-//     then R/16 more tcgen05.mma steps with A = h read straight from tensor
-//     memory and B = the B_cat tile, into the same accumulator; the epilogue
-//     warps convert the tile to bf16 and store it.
-//   * Warp roles: warp 0 issues TMA loads into a 5-stage shared-memory ring
+// Design (persistent; one CTA per SM; clusters of G CTAs share a panel):
+//   * A panel is 128 token rows (one TMEM lane per row).  The G CTAs of a
+//     thread-block cluster work on the same panel at the same time, so the
+//     panel of x is fetched from DRAM once and re-read from L2 by all of them
+//     while they split its N tiles (tile t goes to CTA t mod G).  With G = 1
+//     every SM owns a private panel, which suits small K; for large K the
+//     148 private panels would not fit in L2.
+//   * TMEM (512 columns x 128 lanes) holds the FP32 accumulator of one
+//     128 x 224 output tile in columns [0, 224) and the panel's rank-R
+//     intermediate h = x A_cat^T as packed bf16 pairs in columns
+//     [224, 224 + R/2) -- 288 columns for R = 576.  h never leaves the chip.
+//   * Phase A (per panel): each CTA of the cluster computes its slice of
+//     ceil(R/G) ranks of h (tcgen05.mma, A = x tile, B = A_cat tile, both in
+//     shared memory).  With G = 1 the epilogue writes h straight into TMEM;
+//     with G > 1 each CTA rounds its slice to bf16 into a shared-memory
+//     staging buffer, the CTAs signal each other through cluster-scope
+//     mbarriers, and every CTA copies all G slices (its own and its peers',
+//     through distributed shared memory) into its own TMEM.
+//   * Phase B (per N tile): a K loop x W^T into the accumulator, then R/16
+//     more MMAs with A = h read straight from TMEM and B = the B_cat tile;
+//     the epilogue converts the tile to bf16 and stores it.
+//   * Warp roles: warp 0 issues TMA loads into a ring of 44 KiB stages
 //     (128-byte swizzled K-major tiles), warp 1 issues the MMAs (one thread)
-//     and owns the TMEM allocation, warps 2-5 are the epilogue (each reads
-//     the 32 TMEM lanes its warp may access).
+//     and owns the TMEM allocation, warps 2-9 are the epilogue: each pulls
+//     half of the tile's accumulator into registers, releases the TMEM
+//     accumulator to the next tile's MMAs, then converts and stores y.
 //   * Every mbarrier wait is bounded; on expiry the kernel records
 //     LG_ERR_DEVICE_TIMEOUT in the device error word, drains its own TMA
 //     copies and MMAs, frees its TMEM and returns.
+#include <cstdlib>
 #include <mutex>
 
 #include <cudaTypedefs.h>
@@ -44,37 +53,51 @@ __device__ int g_device_error;
 
 namespace {
 
-constexpr int BM = 128;  // token rows per panel = TMEM lanes
-constexpr int BK = 64;   // K elements per stage: one 128-byte swizzle span
-constexpr int BN = 224;  // output columns per tile
-constexpr int HC = 192;  // rank columns per down-projection chunk
-constexpr int STAGES = 5;
+constexpr int BM = 128;      // token rows per CTA = TMEM lanes
+constexpr int BK = 64;       // K elements per stage: one 128-byte swizzle span
+constexpr int BN = 224;      // output columns per tile
+constexpr int HC_MAX = 192;  // rank columns per down-projection chunk
 constexpr int RMAX = 576;
-constexpr uint32_t A_BYTES = BM * BK * 2;  // 16 KiB: x tile
-constexpr uint32_t B_BYTES = BN * BK * 2;  // 28 KiB: W / A_cat / B_cat tile
-constexpr uint32_t H_TILE_BYTES = HC * BK * 2;
-constexpr uint32_t STAGE_BYTES = A_BYTES + B_BYTES;
+constexpr uint32_t A_BYTES = BM * BK * 2;  // 16 KiB: this CTA's x tile
 constexpr uint32_t TMEM_COLS = 512;
 constexpr uint32_t ACC_COL = 0;
 constexpr uint32_t H_COL = BN;
-constexpr int NUM_THREADS = 192;
+constexpr int NUM_THREADS = 320;  // producer, MMA, 8 epilogue warps
+constexpr int EPI_WARPS = 8;      // two per TMEM lane quarter, one per half tile
+constexpr int HALF_N = BN / 2;    // accumulator columns per epilogue warp
+constexpr int MAX_STAGES = 8;
 constexpr uint64_t TEARDOWN_LIMIT_NS = 200ull * 1000ull * 1000ull;
+constexpr size_t kMaxSmem = 232448;  // sm_100 opt-in maximum per block
 
 static_assert(H_COL + RMAX / 2 <= TMEM_COLS, "h does not fit next to the accumulator");
-static_assert(H_TILE_BYTES <= B_BYTES, "A_cat chunk tile does not fit the B slot");
-static_assert(A_BYTES % 1024 == 0 && STAGE_BYTES % 1024 == 0, "tiles must stay 1024-byte aligned");
+
+// Per-variant constants.  PAIR = false: single-SM tcgen05.mma, 128-row
+// panels, each CTA loads whole B tiles.  PAIR = true: CTA pairs issue
+// tcgen05.mma.cta_group::2 over 256-row panels; each CTA holds 128 rows and
+// loads half of every B tile.
+template <bool PAIR>
+struct Cfg {
+  static constexpr uint32_t B_ROWS = PAIR ? BN / 2 : BN;  // W / B_cat rows a CTA loads
+  static constexpr uint32_t B_BYTES = B_ROWS * BK * 2;
+  static constexpr uint32_t STAGE = A_BYTES + B_BYTES;
+  static constexpr int MMA_M = PAIR ? 2 * BM : BM;
+  static constexpr int PANEL = PAIR ? 2 * BM : BM;
+  static_assert(STAGE % 1024 == 0, "stages must stay 1024-byte aligned");
+  static_assert((PAIR ? HC_MAX / 2 : HC_MAX) * BK * 2 <= B_BYTES, "A_cat chunk tile must fit the B slot");
+};
 
 struct Control {
-  uint64_t full[STAGES];
-  uint64_t empty[STAGES];
-  uint64_t acc_full;
-  uint64_t acc_empty;
-  uint64_t drain;
+  uint64_t full[MAX_STAGES];   // data of a stage has landed (pair: counted on the leader)
+  uint64_t empty[MAX_STAGES];  // the MMAs are done with a stage
+  uint64_t acc_full;           // the tile's accumulator is complete
+  uint64_t acc_empty;          // the epilogue drained the accumulator (pair: on the leader)
+  uint64_t drain;              // every MMA has finished
+  uint64_t slice_ready;        // every group member's slice of h is in its staging rows
+  uint64_t slice_free;         // every group member has copied this CTA's slice
+  uint64_t epi_sync;           // all epilogue warps finished writing this panel's h slice
   uint32_t tmem_base;
   int abort_flag;
 };
-
-constexpr size_t kSmemBytes = 1024 + (size_t)STAGES * STAGE_BYTES + sizeof(Control);
 
 struct Args {
   uint16_t* y;
@@ -83,9 +106,16 @@ struct Args {
   int R;
   int num_panels;
   int n_tiles;
-  int n_chunks;
   int k_blocks;
   int r_blocks;
+  int group;        // members (CTAs, or pairs) sharing one panel
+  int slice;        // ranks of h each member computes (R when group == 1)
+  int n_chunks;     // down-projection chunks per member per panel
+  int chunk_valid;  // ranks per chunk (multiple of 8; the last may hold fewer)
+  int chunk_n;      // MMA N of a chunk: chunk_valid rounded up to 16
+  int stages;
+  uint32_t staging_stride;  // bytes per staging row; the rows live at ring offset 0
+  uint32_t control_off;     // byte offset of the Control block
   unsigned long long wait_limit_ns;
 };
 
@@ -95,13 +125,14 @@ __device__ __forceinline__ void record_timeout(volatile int* abort_flag) {
 }
 
 // Wait for the phase of `bar` with parity `parity` to complete, giving up
-// after limit_ns or as soon as another warp of the CTA has given up.
-__device__ __noinline__ bool wait_bounded(uint32_t bar, uint32_t parity, uint64_t limit_ns,
-                                          volatile int* abort_flag) {
-  if (mbar_try_wait(bar, parity)) return true;
+// after limit_ns or as soon as another warp of the CTA has given up.  With
+// `cluster_scope` the wait acquires at cluster scope (peers' writes made
+// before their release-arrive become visible).
+__device__ __noinline__ bool wait_slow(uint32_t bar, uint32_t parity, uint64_t limit_ns, volatile int* abort_flag,
+                                       bool cluster_scope) {
   const uint64_t t0 = globaltimer_ns();
   for (;;) {
-    if (mbar_try_wait(bar, parity)) return true;
+    if (cluster_scope ? mbar_try_wait_cluster(bar, parity) : mbar_try_wait(bar, parity)) return true;
     if (*abort_flag) return false;
     if (globaltimer_ns() - t0 >= limit_ns) {
       record_timeout(abort_flag);
@@ -109,148 +140,232 @@ __device__ __noinline__ bool wait_bounded(uint32_t bar, uint32_t parity, uint64_
     }
   }
 }
+__device__ __forceinline__ bool wait_bounded(uint32_t bar, uint32_t parity, uint64_t limit_ns,
+                                             volatile int* abort_flag, bool cluster_scope = false) {
+  if (cluster_scope ? mbar_try_wait_cluster(bar, parity) : mbar_try_wait(bar, parity)) return true;
+  return wait_slow(bar, parity, limit_ns, abort_flag, cluster_scope);
+}
 
-// Teardown wait: fixed limit, ignores the abort flag.
-__device__ __noinline__ void wait_teardown(uint32_t bar, uint32_t parity, volatile int* abort_flag) {
+// Teardown wait: ignores the abort flag, gives up after limit_ns.
+__device__ __noinline__ void wait_teardown(uint32_t bar, uint32_t parity, volatile int* abort_flag,
+                                           uint64_t limit_ns = TEARDOWN_LIMIT_NS) {
   if (mbar_try_wait(bar, parity)) return;
   const uint64_t t0 = globaltimer_ns();
   while (!mbar_try_wait(bar, parity)) {
-    if (globaltimer_ns() - t0 >= TEARDOWN_LIMIT_NS) {
+    if (globaltimer_ns() - t0 >= limit_ns) {
       record_timeout(abort_flag);
       return;
     }
   }
 }
 
-__device__ __forceinline__ void advance(uint32_t& stage, uint32_t& phase) {
-  if (++stage == STAGES) {
+__device__ __forceinline__ void fence_proxy_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+__device__ __forceinline__ void advance(uint32_t& stage, uint32_t& phase, uint32_t stages) {
+  if (++stage == stages) {
     stage = 0;
     phase ^= 1;
   }
 }
 
+// Ranks of chunk j of group member `member`: [first, first + count).
+__device__ __forceinline__ void chunk_ranks(const Args& a, int member, int j, int& first, int& count) {
+  const int slice0 = member * a.slice;
+  first = slice0 + j * a.chunk_valid;
+  const int slice_end = min(slice0 + a.slice, a.R);
+  count = max(0, min(a.chunk_valid, slice_end - first));
+}
+
+// ---------------------------------------------------------------------------
+// Producer (warp 0, one thread): TMA loads into the stage ring.  The K sweep
+// alternates direction from one sweep to the next (serpentine order), so the
+// x tiles loaded last are the first ones the next sweep of the same panel
+// re-reads, while they are still in L2.
+// ---------------------------------------------------------------------------
+template <bool PAIR>
 __device__ void run_producer(const CUtensorMap* tm_x, const CUtensorMap* tm_w, const CUtensorMap* tm_a,
                              const CUtensorMap* tm_b, const Args& a, Control* ctl, uint32_t smem_base,
-                             volatile int* abort_flag) {
-  uint32_t stage = 0, phase = 0;
+                             uint32_t crank, uint32_t cid, uint32_t ncl, volatile int* abort_flag) {
+  using C = Cfg<PAIR>;
+  const uint32_t stages = (uint32_t)a.stages;
+  const int member = PAIR ? (int)(crank >> 1) : (int)crank;
+  const int half = PAIR ? (int)(crank & 1) : 0;
+  const bool posts_tx = !PAIR || half == 0;  // the pair leader's barrier counts both CTAs' bytes
+  const uint32_t full_local = smem_u32(&ctl->full[0]);
+  const uint32_t full0 = PAIR ? mapa_shared(full_local, crank & ~1u) : full_local;
+  const uint32_t empty0 = smem_u32(&ctl->empty[0]);
+  const uint32_t slice_free = smem_u32(&ctl->slice_free);
+  const uint32_t a_rows = PAIR ? (uint32_t)a.chunk_n / 2 : (uint32_t)a.chunk_n;
+  const uint32_t mult = PAIR ? 2u : 1u;
+  const uint32_t tx_a = mult * (A_BYTES + a_rows * BK * 2);
+  const uint32_t tx_k = mult * C::STAGE;
+  const uint32_t tx_r = mult * C::B_BYTES;
+  uint32_t stage = 0, phase = 0, sweep = 0, it = 0;
   uint64_t fills = 0;
   bool ok = true;
-  const uint32_t full0 = smem_u32(&ctl->full[0]);
-  const uint32_t empty0 = smem_u32(&ctl->empty[0]);
-  for (int p = blockIdx.x; ok && p < a.num_panels; p += gridDim.x) {
-    const int m0 = p * BM;
-    // Phase A: x panel and A_cat chunks.
-    for (int c = 0; ok && c < a.n_chunks; ++c) {
-      for (int kb = 0; kb < a.k_blocks; ++kb) {
+  auto load = [&](const CUtensorMap* m, uint32_t dst, int c0, int c1) {
+    if constexpr (PAIR) {
+      tma_load_2d_pair(dst, m, full0 + 8 * stage, c0, c1);
+    } else {
+      tma_load_2d(dst, m, full0 + 8 * stage, c0, c1);
+    }
+  };
+  for (int p = (int)cid; ok && p < a.num_panels; p += (int)ncl, ++it) {
+    const int m0 = p * C::PANEL + half * BM;
+    for (int j = 0; ok && j < a.n_chunks; ++j, ++sweep) {
+      int first, count;
+      chunk_ranks(a, member, j, first, count);
+      for (int i = 0; i < a.k_blocks; ++i) {
+        const int kb = (sweep & 1) ? a.k_blocks - 1 - i : i;
         if (!wait_bounded(empty0 + 8 * stage, phase ^ 1, a.wait_limit_ns, abort_flag)) {
           ok = false;
           break;
         }
-        const uint32_t sa = smem_base + stage * STAGE_BYTES;
-        const uint32_t bar = full0 + 8 * stage;
-        mbar_arrive_expect_tx(bar, A_BYTES + H_TILE_BYTES);
-        tma_load_2d(sa, tm_x, bar, kb * BK, m0);
-        tma_load_2d(sa + A_BYTES, tm_a, bar, kb * BK, c * HC);
+        const uint32_t sa = smem_base + stage * C::STAGE;
+        if (posts_tx) mbar_arrive_expect_tx(full_local + 8 * stage, tx_a);
+        load(tm_x, sa, kb * BK, m0);
+        load(tm_a, sa + A_BYTES, kb * BK, first + half * (int)a_rows);
         ++fills;
-        advance(stage, phase);
+        advance(stage, phase, stages);
       }
     }
-    // Phase B: x panel with W, then B_cat for the rank steps.
-    for (int t = 0; ok && t < a.n_tiles; ++t) {
-      const int n0 = t * BN;
-      for (int kb = 0; kb < a.k_blocks; ++kb) {
+    // The h exchange stages this CTA's slice at the start of the ring (idle
+    // once phase A is consumed): hold the phase-B loads until every member of
+    // the group has copied it.
+    if (ok && a.group > 1 && a.R > 0) {
+      ok = wait_bounded(slice_free, it & 1, a.wait_limit_ns, abort_flag, true);
+      fence_proxy_async_smem();
+    }
+    for (int t = member; ok && t < a.n_tiles; t += a.group, ++sweep) {
+      const int n0 = t * BN + half * (int)C::B_ROWS;
+      for (int i = 0; i < a.k_blocks; ++i) {
+        const int kb = (sweep & 1) ? a.k_blocks - 1 - i : i;
         if (!wait_bounded(empty0 + 8 * stage, phase ^ 1, a.wait_limit_ns, abort_flag)) {
           ok = false;
           break;
         }
-        const uint32_t sa = smem_base + stage * STAGE_BYTES;
-        const uint32_t bar = full0 + 8 * stage;
-        mbar_arrive_expect_tx(bar, A_BYTES + B_BYTES);
-        tma_load_2d(sa, tm_x, bar, kb * BK, m0);
-        tma_load_2d(sa + A_BYTES, tm_w, bar, kb * BK, n0);
+        const uint32_t sa = smem_base + stage * C::STAGE;
+        if (posts_tx) mbar_arrive_expect_tx(full_local + 8 * stage, tx_k);
+        load(tm_x, sa, kb * BK, m0);
+        load(tm_w, sa + A_BYTES, kb * BK, n0);
         ++fills;
-        advance(stage, phase);
+        advance(stage, phase, stages);
       }
       for (int rb = 0; ok && rb < a.r_blocks; ++rb) {
         if (!wait_bounded(empty0 + 8 * stage, phase ^ 1, a.wait_limit_ns, abort_flag)) {
           ok = false;
           break;
         }
-        const uint32_t sa = smem_base + stage * STAGE_BYTES;
-        const uint32_t bar = full0 + 8 * stage;
-        mbar_arrive_expect_tx(bar, B_BYTES);
-        tma_load_2d(sa + A_BYTES, tm_b, bar, rb * BK, n0);
+        const uint32_t sa = smem_base + stage * C::STAGE;
+        if (posts_tx) mbar_arrive_expect_tx(full_local + 8 * stage, tx_r);
+        load(tm_b, sa + A_BYTES, rb * BK, n0);
         ++fills;
-        advance(stage, phase);
+        advance(stage, phase, stages);
       }
     }
   }
-  // Let every copy this CTA issued land before the CTA may exit.
-  for (uint32_t s = 0; s < (uint32_t)STAGES; ++s) {
-    const uint64_t fs = fills / STAGES + (s < fills % STAGES ? 1 : 0);
-    if (fs) wait_teardown(full0 + 8 * s, (uint32_t)((fs - 1) & 1), abort_flag);
+  if (posts_tx) {
+    // This CTA's full barriers count every byte loaded for its stages (for a
+    // pair, both CTAs' bytes): once complete, every copy has landed.
+    for (uint32_t s = 0; s < stages; ++s) {
+      const uint64_t fs = fills / stages + (s < fills % stages ? 1 : 0);
+      if (fs) wait_teardown(full_local + 8 * s, (uint32_t)((fs - 1) & 1), abort_flag);
+    }
+  } else if (!ok) {
+    // A pair follower that gave up cannot observe the leader's barriers;
+    // give its copies in flight (microseconds at most) time to land.
+    const uint64_t t0 = globaltimer_ns();
+    while (globaltimer_ns() - t0 < 200000ull) {
+    }
   }
 }
 
-__device__ void run_mma(const Args& a, Control* ctl, uint32_t smem_base, uint32_t tmem,
-                        volatile int* abort_flag) {
+// ---------------------------------------------------------------------------
+// MMA issuer (warp 1, one thread; for pairs only the leader).
+// ---------------------------------------------------------------------------
+template <bool PAIR>
+__device__ void run_mma(const Args& a, Control* ctl, uint32_t smem_base, uint32_t tmem, uint32_t crank, uint32_t cid,
+                        uint32_t ncl, volatile int* abort_flag) {
+  using C = Cfg<PAIR>;
+  const uint32_t stages = (uint32_t)a.stages;
+  const int member = PAIR ? (int)(crank >> 1) : (int)crank;
+  const uint16_t mask = (uint16_t)(3u << (2 * member));
   uint32_t stage = 0, phase = 0, acc_phase = 0;
   bool ok = true;
   const uint32_t full0 = smem_u32(&ctl->full[0]);
   const uint32_t empty0 = smem_u32(&ctl->empty[0]);
   const uint32_t acc_full = smem_u32(&ctl->acc_full);
   const uint32_t acc_empty = smem_u32(&ctl->acc_empty);
-  constexpr uint32_t idesc_h = idesc_bf16_f32(BM, HC);
-  constexpr uint32_t idesc_y = idesc_bf16_f32(BM, BN);
+  const uint32_t idesc_h = idesc_bf16_f32(C::MMA_M, a.chunk_n);
+  constexpr uint32_t idesc_y = idesc_bf16_f32(C::MMA_M, BN);
   const uint32_t d_acc = tmem + ACC_COL;
-  for (int p = blockIdx.x; ok && p < a.num_panels; p += gridDim.x) {
-    for (int c = 0; ok && c < a.n_chunks; ++c) {
-      if (!wait_bounded(acc_empty, acc_phase ^ 1, a.wait_limit_ns, abort_flag)) {
+  auto commit = [&](uint32_t bar) {
+    if constexpr (PAIR) {
+      umma_commit_pair_mc(bar, mask);
+    } else {
+      umma_commit(bar);
+    }
+  };
+  auto mma_ss = [&](uint64_t da, uint64_t db, uint32_t idesc, uint32_t acc) {
+    if constexpr (PAIR) {
+      umma_ss_pair(d_acc, da, db, idesc, acc);
+    } else {
+      umma_ss(d_acc, da, db, idesc, acc);
+    }
+  };
+  auto mma_ts = [&](uint32_t a_tmem, uint64_t db) {
+    if constexpr (PAIR) {
+      umma_ts_pair(d_acc, a_tmem, db, idesc_y, 1u);
+    } else {
+      umma_ts(d_acc, a_tmem, db, idesc_y, 1u);
+    }
+  };
+  for (int p = (int)cid; ok && p < a.num_panels; p += (int)ncl) {
+    for (int j = 0; ok && j < a.n_chunks; ++j) {
+      if (!wait_bounded(acc_empty, acc_phase ^ 1, a.wait_limit_ns, abort_flag, PAIR)) {
         ok = false;
         break;
       }
       tc_fence_after();
-      for (int kb = 0; kb < a.k_blocks; ++kb) {
+      for (int i = 0; i < a.k_blocks; ++i) {
         if (!wait_bounded(full0 + 8 * stage, phase, a.wait_limit_ns, abort_flag)) {
           ok = false;
           break;
         }
         tc_fence_after();
-        const uint32_t sa = smem_base + stage * STAGE_BYTES;
+        const uint32_t sa = smem_base + stage * C::STAGE;
         const uint64_t da = sw128_kmajor_desc(sa);
         const uint64_t db = sw128_kmajor_desc(sa + A_BYTES);
 #pragma unroll
-        for (int kk = 0; kk < BK / 16; ++kk) {
-          umma_ss(d_acc, da + 2 * kk, db + 2 * kk, idesc_h, (kb | kk) != 0);
-        }
-        umma_commit(empty0 + 8 * stage);
-        advance(stage, phase);
+        for (int kk = 0; kk < BK / 16; ++kk) mma_ss(da + 2 * kk, db + 2 * kk, idesc_h, (i | kk) != 0);
+        commit(empty0 + 8 * stage);
+        advance(stage, phase, stages);
       }
       if (!ok) break;
-      umma_commit(acc_full);
+      commit(acc_full);
       acc_phase ^= 1;
     }
-    for (int t = 0; ok && t < a.n_tiles; ++t) {
-      if (!wait_bounded(acc_empty, acc_phase ^ 1, a.wait_limit_ns, abort_flag)) {
+    for (int t = member; ok && t < a.n_tiles; t += a.group) {
+      if (!wait_bounded(acc_empty, acc_phase ^ 1, a.wait_limit_ns, abort_flag, PAIR)) {
         ok = false;
         break;
       }
       tc_fence_after();
-      for (int kb = 0; kb < a.k_blocks; ++kb) {
+      for (int i = 0; i < a.k_blocks; ++i) {
         if (!wait_bounded(full0 + 8 * stage, phase, a.wait_limit_ns, abort_flag)) {
           ok = false;
           break;
         }
         tc_fence_after();
-        const uint32_t sa = smem_base + stage * STAGE_BYTES;
+        const uint32_t sa = smem_base + stage * C::STAGE;
         const uint64_t da = sw128_kmajor_desc(sa);
         const uint64_t db = sw128_kmajor_desc(sa + A_BYTES);
 #pragma unroll
-        for (int kk = 0; kk < BK / 16; ++kk) {
-          umma_ss(d_acc, da + 2 * kk, db + 2 * kk, idesc_y, (kb | kk) != 0);
-        }
-        umma_commit(empty0 + 8 * stage);
-        advance(stage, phase);
+        for (int kk = 0; kk < BK / 16; ++kk) mma_ss(da + 2 * kk, db + 2 * kk, idesc_y, (i | kk) != 0);
+        commit(empty0 + 8 * stage);
+        advance(stage, phase, stages);
       }
       for (int rb = 0; ok && rb < a.r_blocks; ++rb) {
         if (!wait_bounded(full0 + 8 * stage, phase, a.wait_limit_ns, abort_flag)) {
@@ -258,106 +373,238 @@ __device__ void run_mma(const Args& a, Control* ctl, uint32_t smem_base, uint32_
           break;
         }
         tc_fence_after();
-        const uint32_t sa = smem_base + stage * STAGE_BYTES;
+        const uint32_t sa = smem_base + stage * C::STAGE;
         const uint64_t db = sw128_kmajor_desc(sa + A_BYTES);
 #pragma unroll
         for (int kk = 0; kk < BK / 16; ++kk) {
           // 16 ranks of h = 8 packed columns.
-          umma_ts(d_acc, tmem + H_COL + (uint32_t)(rb * (BK / 2) + kk * 8), db + 2 * kk, idesc_y, 1u);
+          mma_ts(tmem + H_COL + (uint32_t)(rb * (BK / 2) + kk * 8), db + 2 * kk);
         }
-        umma_commit(empty0 + 8 * stage);
-        advance(stage, phase);
+        commit(empty0 + 8 * stage);
+        advance(stage, phase, stages);
       }
       if (!ok) break;
-      umma_commit(acc_full);
+      commit(acc_full);
       acc_phase ^= 1;
     }
   }
-  // Every MMA this thread issued must finish before TMEM is freed.
-  const uint32_t drain = smem_u32(&ctl->drain);
-  umma_commit(drain);
-  wait_teardown(drain, 0, abort_flag);
+  // Every MMA must finish before TMEM is freed or (for a pair) either CTA exits.
+  commit(smem_u32(&ctl->drain));
+  wait_teardown(smem_u32(&ctl->drain), 0, abort_flag);
 }
 
-__device__ void run_epilogue(const Args& a, Control* ctl, uint32_t tmem, int warp, int lane,
-                             volatile int* abort_flag) {
-  const int q = warp & 3;  // TMEM lanes 32q .. 32q+31 belong to this warp
+// ---------------------------------------------------------------------------
+// Epilogue helpers (one warp: TMEM lanes of its quarter, half of the blocks).
+// ---------------------------------------------------------------------------
+// FP32 accumulator columns [0, count) = ranks first .. first+count-1 ->
+// bf16 pairs in the h columns.  count is a multiple of 8.
+__device__ __forceinline__ void acc_to_h(uint32_t lane_base, int first, int count, int half) {
+  const int full_blocks = count / 16;
+  for (int b = half; b < full_blocks; b += 2) {
+    uint32_t v[16];
+    tmem_ld_32x32b_x16(lane_base + ACC_COL + 16 * b, v);
+    tmem_wait_ld();
+    uint32_t packed[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) packed[i] = pack_bf16x2(__uint_as_float(v[2 * i]), __uint_as_float(v[2 * i + 1]));
+    tmem_st_32x32b_x8(lane_base + H_COL + (uint32_t)((first + 16 * b) / 2), packed);
+  }
+  if ((count % 16) && ((full_blocks & 1) == half)) {
+    uint32_t v[8];
+    tmem_ld_32x32b_x8(lane_base + ACC_COL + 16 * full_blocks, v);
+    tmem_wait_ld();
+    uint32_t packed[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) packed[i] = pack_bf16x2(__uint_as_float(v[2 * i]), __uint_as_float(v[2 * i + 1]));
+    tmem_st_32x32b_x4(lane_base + H_COL + (uint32_t)((first + 16 * full_blocks) / 2), packed);
+  }
+  tmem_wait_st();
+}
+
+// This member's slice of h (pairs s0/2 .. ) from TMEM into its staging row.
+__device__ __forceinline__ void h_to_staging(uint32_t lane_base, int s0, int slice, int half, uint32_t row) {
+  const int cols = slice / 2;  // multiple of 4
+  const uint32_t src = lane_base + H_COL + (uint32_t)(s0 / 2);
+  for (int b = half; b < cols / 8; b += 2) {
+    uint32_t v[8];
+    tmem_ld_32x32b_x8(src + 8 * b, v);
+    tmem_wait_ld();
+    st_shared_v4(row + 32u * b, v[0], v[1], v[2], v[3]);
+    st_shared_v4(row + 32u * b + 16, v[4], v[5], v[6], v[7]);
+  }
+  if ((cols % 8) && (((cols / 8) & 1) == half)) {
+    uint32_t v[4];
+    tmem_ld_32x32b_x4(src + 8 * (cols / 8), v);
+    tmem_wait_ld();
+    st_shared_v4(row + 32u * (cols / 8), v[0], v[1], v[2], v[3]);
+  }
+}
+
+// A peer's staged slice (cluster address of its row) into this CTA's h columns.
+__device__ __forceinline__ void staging_to_h(uint32_t lane_base, int s0, int slice, int half, uint32_t remote_row) {
+  const int cols = slice / 2;
+  const uint32_t dst = lane_base + H_COL + (uint32_t)(s0 / 2);
+  for (int b = half; b < cols / 8; b += 2) {
+    uint32_t v[8];
+    ld_shared_cluster_v4(remote_row + 32u * b, v[0], v[1], v[2], v[3]);
+    ld_shared_cluster_v4(remote_row + 32u * b + 16, v[4], v[5], v[6], v[7]);
+    tmem_st_32x32b_x8(dst + 8 * b, v);
+  }
+  if ((cols % 8) && (((cols / 8) & 1) == half)) {
+    uint32_t v[4];
+    ld_shared_cluster_v4(remote_row + 32u * (cols / 8), v[0], v[1], v[2], v[3]);
+    tmem_st_32x32b_x4(dst + 8 * (cols / 8), v);
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Epilogue (warps 2..9): warp w reads TMEM lanes 32 (w mod 4) .. +31 and
+// handles half (w - 2) / 4 of the columns.
+// ---------------------------------------------------------------------------
+template <bool PAIR>
+__device__ void run_epilogue(const Args& a, Control* ctl, uint32_t smem_base, uint32_t tmem, uint32_t crank,
+                             uint32_t cid, uint32_t ncl, int warp, int lane, volatile int* abort_flag) {
+  using C = Cfg<PAIR>;
+  const int q = warp & 3;
+  const int half = (warp - 2) >> 2;
+  const int parity = PAIR ? (int)(crank & 1) : 0;
+  const int member = PAIR ? (int)(crank >> 1) : (int)crank;
+  const int row_in_tile = 32 * q + lane;
   const uint32_t lane_base = tmem + ((uint32_t)(32 * q) << 16);
   const uint32_t acc_full = smem_u32(&ctl->acc_full);
-  const uint32_t acc_empty = smem_u32(&ctl->acc_empty);
+  const uint32_t acc_empty = PAIR ? mapa_shared(smem_u32(&ctl->acc_empty), crank & ~1u) : smem_u32(&ctl->acc_empty);
+  const uint32_t slice_ready = smem_u32(&ctl->slice_ready);
+  const uint32_t slice_free = smem_u32(&ctl->slice_free);
+  const uint32_t epi_sync = smem_u32(&ctl->epi_sync);
+  const uint32_t my_row = smem_base + (uint32_t)row_in_tile * a.staging_stride;
+  auto peer_rank = [&](int c) { return (uint32_t)(PAIR ? 2 * c + parity : c); };
   uint32_t acc_phase = 0;
+  uint32_t it = 0;
   bool ok = true;
-  for (int p = blockIdx.x; ok && p < a.num_panels; p += gridDim.x) {
-    const int64_t m0 = (int64_t)p * BM;
-    for (int c = 0; ok && c < a.n_chunks; ++c) {
-      ok = __all_sync(0xffffffffu, wait_bounded(acc_full, acc_phase, a.wait_limit_ns, abort_flag));
-      if (!ok) break;
-      tc_fence_after();
-      const int valid = min(HC, a.R - c * HC);
-      for (int j = 0; j < valid / 32; ++j) {
-        uint32_t v[32];
-        tmem_ld_32x32b_x32(lane_base + ACC_COL + 32 * j, v);
-        tmem_wait_ld();
-        uint32_t packed[16];
-#pragma unroll
-        for (int i = 0; i < 16; ++i) packed[i] = pack_bf16x2(__uint_as_float(v[2 * i]), __uint_as_float(v[2 * i + 1]));
-        tmem_st_32x32b_x16(lane_base + H_COL + (uint32_t)((c * HC + 32 * j) / 2), packed);
+  auto release_acc = [&]() {
+    tc_fence_before();
+    __syncwarp();
+    if (lane == 0) {
+      if constexpr (PAIR) {
+        mbar_arrive_remote(acc_empty);
+      } else {
+        mbar_arrive(acc_empty);
       }
-      tmem_wait_st();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(acc_empty);
-      acc_phase ^= 1;
     }
-    for (int t = 0; ok && t < a.n_tiles; ++t) {
+    acc_phase ^= 1;
+  };
+  for (int p = (int)cid; ok && p < a.num_panels; p += (int)ncl, ++it) {
+    const int64_t m0 = (int64_t)p * C::PANEL + parity * BM;
+    for (int j = 0; ok && j < a.n_chunks; ++j) {
       ok = __all_sync(0xffffffffu, wait_bounded(acc_full, acc_phase, a.wait_limit_ns, abort_flag));
       if (!ok) break;
       tc_fence_after();
-      const int64_t row = m0 + 32 * q + lane;
-      const int n0 = t * BN;
-      for (int j = 0; j < BN / 32; ++j) {
-        uint32_t v[32];
-        tmem_ld_32x32b_x32(lane_base + ACC_COL + 32 * j, v);
-        tmem_wait_ld();
-        const int col = n0 + 32 * j;
-        if (row < a.M && col < a.N) {
-          uint4* dst = reinterpret_cast<uint4*>(a.y + row * (int64_t)a.N + col);
-#pragma unroll
-          for (int g = 0; g < 4; ++g) {
-            dst[g] = make_uint4(pack_bf16x2(__uint_as_float(v[8 * g + 0]), __uint_as_float(v[8 * g + 1])),
-                                pack_bf16x2(__uint_as_float(v[8 * g + 2]), __uint_as_float(v[8 * g + 3])),
-                                pack_bf16x2(__uint_as_float(v[8 * g + 4]), __uint_as_float(v[8 * g + 5])),
-                                pack_bf16x2(__uint_as_float(v[8 * g + 6]), __uint_as_float(v[8 * g + 7])));
-          }
+      int first, count;
+      chunk_ranks(a, member, j, first, count);
+      acc_to_h(lane_base, first, count, half);
+      if (a.group > 1 && j == a.n_chunks - 1) {
+        // Swap slices with the other members of the group: stage this slice
+        // at the start of the (idle) ring, wait for every member's, copy the
+        // peers' slices into TMEM, then release the staging rows.  The two
+        // warps of a lane quarter first agree that the slice is complete in
+        // TMEM (a block may be staged by the warp that did not write it).
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(epi_sync);
+        ok = __all_sync(0xffffffffu, wait_bounded(epi_sync, it & 1, a.wait_limit_ns, abort_flag));
+        if (!ok) break;
+        tc_fence_after();
+        fence_proxy_async_smem();
+        h_to_staging(lane_base, member * a.slice, a.slice, half, my_row);
+        __syncwarp();
+        if (lane == 0) {
+          for (int c = 0; c < a.group; ++c) mbar_arrive_remote(mapa_shared(slice_ready, peer_rank(c)));
+        }
+        ok = __all_sync(0xffffffffu, wait_bounded(slice_ready, it & 1, a.wait_limit_ns, abort_flag, true));
+        if (!ok) break;
+        for (int c = 0; c < a.group; ++c) {
+          if (c != member) staging_to_h(lane_base, c * a.slice, a.slice, half, mapa_shared(my_row, peer_rank(c)));
+        }
+        tmem_wait_st();
+        __syncwarp();
+        if (lane == 0) {
+          for (int c = 0; c < a.group; ++c) mbar_arrive_remote(mapa_shared(slice_free, peer_rank(c)));
         }
       }
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(acc_empty);
-      acc_phase ^= 1;
+      release_acc();
+    }
+    for (int t = member; ok && t < a.n_tiles; t += a.group) {
+      ok = __all_sync(0xffffffffu, wait_bounded(acc_full, acc_phase, a.wait_limit_ns, abort_flag));
+      if (!ok) break;
+      tc_fence_after();
+      // Pull this warp's 112 accumulator columns into registers and hand the
+      // accumulator back at once, so the next tile's MMAs overlap the
+      // conversion and the stores below.
+      const uint32_t src = lane_base + ACC_COL + (uint32_t)(half * HALF_N);
+      uint32_t v0[32], v1[32], v2[32], v3[16];
+      tmem_ld_32x32b_x32(src, v0);
+      tmem_ld_32x32b_x32(src + 32, v1);
+      tmem_ld_32x32b_x32(src + 64, v2);
+      tmem_ld_32x32b_x16(src + 96, v3);
+      tmem_wait_ld();
+      release_acc();
+
+      const int64_t row = m0 + row_in_tile;
+      const int col0 = t * BN + half * HALF_N;
+      if (row < a.M) {
+        uint16_t* dst_row = a.y + row * (int64_t)a.N;
+        auto store8 = [&](int g, const uint32_t* v) {
+          const int col = col0 + 8 * g;
+          if (col < a.N) {
+            *reinterpret_cast<uint4*>(dst_row + col) =
+                make_uint4(pack_bf16x2(__uint_as_float(v[0]), __uint_as_float(v[1])),
+                           pack_bf16x2(__uint_as_float(v[2]), __uint_as_float(v[3])),
+                           pack_bf16x2(__uint_as_float(v[4]), __uint_as_float(v[5])),
+                           pack_bf16x2(__uint_as_float(v[6]), __uint_as_float(v[7])));
+          }
+        };
+#pragma unroll
+        for (int g = 0; g < 4; ++g) store8(g, v0 + 8 * g);
+#pragma unroll
+        for (int g = 0; g < 4; ++g) store8(4 + g, v1 + 8 * g);
+#pragma unroll
+        for (int g = 0; g < 4; ++g) store8(8 + g, v2 + 8 * g);
+#pragma unroll
+        for (int g = 0; g < 2; ++g) store8(12 + g, v3 + 8 * g);
+      }
     }
   }
 }
 
+template <bool PAIR>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     k_lora_linear(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_w,
                   const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b,
                   const Args args) {
   extern __shared__ uint8_t smem_raw[];
+  // Dynamic shared memory starts at the same offset in every CTA, so after
+  // rounding up to 1 KiB the layout (and every mapa'd address) matches.
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
-  Control* ctl = reinterpret_cast<Control*>(smem + (size_t)STAGES * STAGE_BYTES);
+  Control* ctl = reinterpret_cast<Control*>(smem + args.control_off);
   const int warp = threadIdx.x / 32;
   const int lane = threadIdx.x % 32;
   const uint32_t smem_base = smem_u32(smem);
+  const uint32_t crank = cluster_ctarank();
+  const uint32_t cid = cluster_id_x();
+  const uint32_t ncl = cluster_count_x();
+  const bool issues_mma = !PAIR || (crank & 1) == 0;
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < STAGES; ++s) {
+    for (int s = 0; s < args.stages; ++s) {
       mbar_init(smem_u32(&ctl->full[s]), 1);
       mbar_init(smem_u32(&ctl->empty[s]), 1);
     }
     mbar_init(smem_u32(&ctl->acc_full), 1);
-    mbar_init(smem_u32(&ctl->acc_empty), 4);
+    mbar_init(smem_u32(&ctl->acc_empty), PAIR ? 2 * EPI_WARPS : EPI_WARPS);
     mbar_init(smem_u32(&ctl->drain), 1);
+    mbar_init(smem_u32(&ctl->slice_ready), EPI_WARPS * args.group);
+    mbar_init(smem_u32(&ctl->slice_free), EPI_WARPS * args.group);
+    mbar_init(smem_u32(&ctl->epi_sync), EPI_WARPS);
     ctl->abort_flag = 0;
     fence_mbarrier_init();
     tma_prefetch_desc(&tm_x);
@@ -368,31 +615,53 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     }
   }
   if (warp == 1) {
-    tmem_alloc(smem_u32(&ctl->tmem_base), TMEM_COLS);
-    tmem_relinquish();
+    if constexpr (PAIR) {
+      tmem_alloc_pair(smem_u32(&ctl->tmem_base), TMEM_COLS);
+      tmem_relinquish_pair();
+    } else {
+      tmem_alloc(smem_u32(&ctl->tmem_base), TMEM_COLS);
+      tmem_relinquish();
+    }
     tc_fence_before();
   }
-  __syncthreads();
+  // Peers may arrive on this CTA's barriers only after they are initialised.
+  cluster_sync_all();
   tc_fence_after();
   const uint32_t tmem = ctl->tmem_base;
   volatile int* abort_flag = &ctl->abort_flag;
 
   if (warp == 0) {
-    if (lane == 0) run_producer(&tm_x, &tm_w, &tm_a, &tm_b, args, ctl, smem_base, abort_flag);
+    if (lane == 0) run_producer<PAIR>(&tm_x, &tm_w, &tm_a, &tm_b, args, ctl, smem_base, crank, cid, ncl, abort_flag);
     __syncwarp();
   } else if (warp == 1) {
-    if (lane == 0) run_mma(args, ctl, smem_base, tmem, abort_flag);
+    if (lane == 0 && issues_mma) run_mma<PAIR>(args, ctl, smem_base, tmem, crank, cid, ncl, abort_flag);
     __syncwarp();
   } else {
-    run_epilogue(args, ctl, tmem, warp, lane, abort_flag);
+    run_epilogue<PAIR>(args, ctl, smem_base, tmem, crank, cid, ncl, warp, lane, abort_flag);
   }
 
   tc_fence_before();
   __syncthreads();
+  if constexpr (PAIR) {
+    // The leader's MMAs read this CTA's shared memory and write its TMEM: the
+    // follower waits for the leader's final (multicast) drain commit.  Its own
+    // epilogue is finished, so at most one wait limit remains on the leader.
+    if (!issues_mma && warp == 1 && lane == 0) {
+      wait_teardown(smem_u32(&ctl->drain), 0, abort_flag, args.wait_limit_ns + TEARDOWN_LIMIT_NS);
+    }
+  }
+  // Every CTA of the cluster is past its last TMEM and shared-memory access
+  // by peers before any frees TMEM or exits.
+  cluster_sync_all();
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tmem, TMEM_COLS);
+    if constexpr (PAIR) {
+      tmem_dealloc_pair(tmem, TMEM_COLS);
+    } else {
+      tmem_dealloc(tmem, TMEM_COLS);
+    }
   }
+  cluster_sync_all();
 }
 
 PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
@@ -422,21 +691,105 @@ bool make_map(PFN_cuTensorMapEncodeTiled_v12000 enc, CUtensorMap* m, const void*
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-}  // namespace
+// Launch geometry: down-projection chunking and stage count.  The h
+// exchange of a group reuses the start of the stage ring, so every stage of
+// shared memory goes to the ring.
+struct Geometry {
+  int group = 1, slice = 0, n_chunks = 0, chunk_valid = 0, chunk_n = 16, stages = 0;
+  uint32_t staging_stride = 0, control_off = 0;
+  size_t smem = 0;
+};
 
-cudaError_t launch_lora_linear(const LinearLaunch& p, cudaStream_t s, bool* driver_failed) {
-  *driver_failed = false;
-  PFN_cuTensorMapEncodeTiled_v12000 enc = tensor_map_encoder();
-  if (!enc) {
-    *driver_failed = true;
-    return cudaErrorNotSupported;
+template <bool PAIR>
+bool make_geometry(int group, int R, Geometry* g) {
+  using C = Cfg<PAIR>;
+  g->group = group;
+  if (R > 0) {
+    if (R % group) return false;
+    g->slice = R / group;
+    if (g->slice % 8) return false;
+    g->n_chunks = (g->slice + HC_MAX - 1) / HC_MAX;
+    g->chunk_valid = ((g->slice + g->n_chunks - 1) / g->n_chunks + 7) / 8 * 8;
+    g->chunk_n = (g->chunk_valid + 15) / 16 * 16;
+    if (g->chunk_n > HC_MAX) return false;
+    g->staging_stride = (uint32_t)(2 * g->slice + 16);
   }
+  const size_t fixed = 1024 + sizeof(Control);
+  g->stages = (int)((kMaxSmem - fixed) / C::STAGE);
+  if (g->stages > MAX_STAGES) g->stages = MAX_STAGES;
+  if (g->stages < 2) return false;
+  if (group > 1 && (size_t)BM * g->staging_stride > (size_t)g->stages * C::STAGE) return false;
+  g->control_off = (uint32_t)g->stages * C::STAGE;
+  g->smem = 1024 + (size_t)g->control_off + sizeof(Control);
+  return true;
+}
+
+int g_cluster_override = 0;  // 0: automatic (lg_set_cluster_size)
+int g_variant_override = 0;  // 0: automatic, 1: single-SM MMA, 2: SM-pair MMA
+
+// Resident clusters of `cluster` CTAs of `kernel` on device `dev` (cached).
+int max_active_clusters(const void* kernel, int variant, int dev, int cluster, size_t smem, int sm_count) {
+  static std::mutex mu;
+  struct Entry {
+    bool known = false;
+    int n = 0;
+  };
+  static Entry cache[64][2][17];
+  std::lock_guard<std::mutex> lock(mu);
+  Entry* en = (dev >= 0 && dev < 64 && cluster <= 16) ? &cache[dev][variant - 1][cluster] : nullptr;
+  if (en && en->known) return en->n;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)(cluster * sm_count), 1, 1);
+  cfg.blockDim = dim3(NUM_THREADS, 1, 1);
+  cfg.dynamicSmemBytes = smem;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = (unsigned)cluster;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  int n = 0;
+  if (cudaOccupancyMaxActiveClusters(&n, kernel, &cfg) != cudaSuccess) {
+    cudaGetLastError();
+    n = 0;
+  }
+  if (en) {
+    en->known = true;
+    en->n = n;
+  }
+  return n;
+}
+
+cudaError_t configure_kernels(int dev) {
+  static std::mutex mu;
+  static bool configured[64] = {};
+  std::lock_guard<std::mutex> lock(mu);
+  if (dev >= 0 && dev < 64 && configured[dev]) return cudaSuccess;
+  const void* kernels[2] = {(const void*)k_lora_linear<false>, (const void*)k_lora_linear<true>};
+  for (const void* k : kernels) {
+    cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kMaxSmem);
+    if (e == cudaSuccess) e = cudaFuncSetAttribute(k, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+    if (e != cudaSuccess) return e;
+  }
+  if (dev >= 0 && dev < 64) configured[dev] = true;
+  return cudaSuccess;
+}
+
+template <bool PAIR>
+cudaError_t launch_variant(const LinearLaunch& p, cudaStream_t s, int dev, int cluster, bool* driver_failed,
+                           PFN_cuTensorMapEncodeTiled_v12000 enc) {
+  using C = Cfg<PAIR>;
+  const int group = PAIR ? cluster / 2 : cluster;
+  Geometry geo;
+  if (!make_geometry<PAIR>(group, p.R, &geo)) return cudaErrorInvalidConfiguration;
+  const uint32_t a_rows = PAIR ? (uint32_t)geo.chunk_n / 2 : (uint32_t)geo.chunk_n;
   CUtensorMap tm_x, tm_w, tm_a, tm_b;
   bool ok = make_map(enc, &tm_x, p.x, (uint64_t)p.K, (uint64_t)p.M, BM) &&
-            make_map(enc, &tm_w, p.W, (uint64_t)p.K, (uint64_t)p.N, BN);
+            make_map(enc, &tm_w, p.W, (uint64_t)p.K, (uint64_t)p.N, C::B_ROWS);
   if (ok && p.R > 0) {
-    ok = make_map(enc, &tm_a, p.A_bf16, (uint64_t)p.K, (uint64_t)p.R, HC) &&
-         make_map(enc, &tm_b, p.B_bf16, (uint64_t)p.R, (uint64_t)p.N, BN);
+    ok = make_map(enc, &tm_a, p.A_bf16, (uint64_t)p.K, (uint64_t)p.R, a_rows) &&
+         make_map(enc, &tm_b, p.B_bf16, (uint64_t)p.R, (uint64_t)p.N, C::B_ROWS);
   } else {
     tm_a = tm_x;  // never read when R == 0
     tm_b = tm_x;
@@ -445,35 +798,76 @@ cudaError_t launch_lora_linear(const LinearLaunch& p, cudaStream_t s, bool* driv
     *driver_failed = true;
     return cudaErrorInvalidValue;
   }
-
-  static std::mutex mu;
-  static bool configured[64] = {};
-  int dev = 0;
-  cudaError_t e = cudaGetDevice(&dev);
-  if (e != cudaSuccess) return e;
-  {
-    std::lock_guard<std::mutex> lock(mu);
-    if (dev < 0 || dev >= 64 || !configured[dev]) {
-      e = cudaFuncSetAttribute(k_lora_linear, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBytes);
-      if (e != cudaSuccess) return e;
-      if (dev >= 0 && dev < 64) configured[dev] = true;
-    }
-  }
-
   Args args;
   args.y = reinterpret_cast<uint16_t*>(p.y);
   args.M = p.M;
   args.N = p.N;
   args.R = p.R;
-  args.num_panels = (int)((p.M + BM - 1) / BM);
+  args.num_panels = (int)((p.M + C::PANEL - 1) / C::PANEL);
   args.n_tiles = (p.N + BN - 1) / BN;
-  args.n_chunks = (p.R + HC - 1) / HC;
   args.k_blocks = p.K / BK;
   args.r_blocks = p.R / BK;
+  args.group = group;
+  args.slice = geo.slice;
+  args.n_chunks = geo.n_chunks;
+  args.chunk_valid = geo.chunk_valid;
+  args.chunk_n = geo.chunk_n;
+  args.stages = geo.stages;
+  args.staging_stride = geo.staging_stride;
+  args.control_off = geo.control_off;
   args.wait_limit_ns = p.wait_limit_ns;
-  const int grid = args.num_panels < p.sm_count ? args.num_panels : p.sm_count;
-  k_lora_linear<<<grid, NUM_THREADS, kSmemBytes, s>>>(tm_x, tm_w, tm_a, tm_b, args);
+  const void* kernel = (const void*)k_lora_linear<PAIR>;
+  int clusters = max_active_clusters(kernel, PAIR ? 2 : 1, dev, cluster, geo.smem, p.sm_count);
+  if (clusters <= 0) clusters = p.sm_count / cluster;
+  if (clusters > args.num_panels) clusters = args.num_panels;
+  if (clusters < 1) clusters = 1;
+
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)(clusters * cluster), 1, 1);
+  cfg.blockDim = dim3(NUM_THREADS, 1, 1);
+  cfg.dynamicSmemBytes = geo.smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = (unsigned)cluster;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  void* params[5] = {&tm_x, &tm_w, &tm_a, &tm_b, &args};
+  cudaError_t e = cudaLaunchKernelExC(&cfg, kernel, params);
+  if (e != cudaSuccess) return e;
   return cudaGetLastError();
+}
+
+}  // namespace
+
+void set_cluster_override(int g) { g_cluster_override = g; }
+void set_variant_override(int v) { g_variant_override = v; }
+
+cudaError_t launch_lora_linear(const LinearLaunch& p, cudaStream_t s, bool* driver_failed) {
+  *driver_failed = false;
+  PFN_cuTensorMapEncodeTiled_v12000 enc = tensor_map_encoder();
+  if (!enc) {
+    *driver_failed = true;
+    return cudaErrorNotSupported;
+  }
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  e = configure_kernels(dev);
+  if (e != cudaSuccess) return e;
+  // Variant and cluster size (both process-wide overrides for tuning).
+  const int variant = g_variant_override ? g_variant_override : 1;
+  int cluster = g_cluster_override;
+  if (variant == 1) {
+    if (cluster == 0) cluster = p.K <= 2048 ? 1 : 2;
+    if (cluster > 8) cluster = 8;
+    return launch_variant<false>(p, s, dev, cluster, driver_failed, enc);
+  }
+  if (cluster < 2) cluster = 2;
+  if (cluster > 8) cluster = 8;
+  return launch_variant<true>(p, s, dev, cluster, driver_failed, enc);
 }
 
 cudaError_t read_and_clear_device_error(cudaStream_t s, int* value) {

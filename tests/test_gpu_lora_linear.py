@@ -140,3 +140,70 @@ def test_wait_timeout_is_reported_and_context_survives():
     y = lg.lora_linear(x, W, A, B)
     err = _check(x, W, A, B, y)
     assert err <= TOL, err
+
+
+@pytest.mark.parametrize("variant,G", [(1, 1), (1, 2), (1, 4), (1, 8), (2, 2), (2, 4), (2, 8)])
+@pytest.mark.parametrize(
+    "M,K,N,R",
+    [
+        (517, 320, 320, 576),    # ragged M and N, full rank, fewer N tiles than CTAs for G >= 4
+        (1000, 1024, 896, 64),   # small rank: slices of 64 / 32 / 16 / 8 ranks
+        (300, 256, 1568, 0),     # no LoRA: the cluster only splits N tiles
+        (2304, 1024, 1024, 576),
+        (37 * 128 + 5, 512, 3584, 576),  # more panels than resident clusters
+    ],
+)
+def test_cluster_sizes(variant, G, M, K, N, R):
+    """Every variant and cluster size: CTAs of a cluster share a panel and
+    exchange their slices of h; SM pairs split every B tile."""
+    x, W, A, B = _rand_layer(M, K, N, R, seed=G * 1000 + M)
+    lg.set_kernel_variant(variant)
+    lg.set_cluster_size(G)
+    try:
+        y = lg.lora_linear(x, W, A if R else None, B if R else None)
+        err = _check(x, W, A, B, y)
+    finally:
+        lg.set_cluster_size(0)
+        lg.set_kernel_variant(0)
+    assert err <= TOL, err
+
+
+@pytest.mark.parametrize("variant,G", [(1, 4), (2, 2), (2, 4)])
+def test_wait_timeout_with_clusters(variant, G):
+    x, W, A, B = _rand_layer(2048, 1024, 1792, 576, seed=19)
+    lg.set_kernel_variant(variant)
+    lg.set_cluster_size(G)
+    lg.set_wait_limit_ns(1)
+    try:
+        lg.lora_linear(x, W, A, B)
+        status = lg.get_last_device_error()
+    finally:
+        lg.set_wait_limit_ns(0)
+    try:
+        assert status == lg.LG_ERR_DEVICE_TIMEOUT
+        y = lg.lora_linear(x, W, A, B)
+        err = _check(x, W, A, B, y)
+    finally:
+        lg.set_cluster_size(0)
+        lg.set_kernel_variant(0)
+    assert err <= TOL, err
+
+
+@pytest.mark.parametrize("name,layer", [("768p", 0), ("2k", 0), ("2k", 2)])
+def test_full_size_sampled_rows_pair_variant(name, layer):
+    lg.set_kernel_variant(2)
+    try:
+        err = _sampled_rows_case(name, layer)
+    finally:
+        lg.set_kernel_variant(0)
+    assert err <= TOL, err
+
+
+def test_cluster_size_argument_checked():
+    with pytest.raises(lg.LoraGemmError) as ei:
+        lg.set_cluster_size(3)
+    assert ei.value.status == lg.LG_ERR_INVALID_ARG
+    with pytest.raises(lg.LoraGemmError):
+        lg.set_cluster_size(16)
+    with pytest.raises(lg.LoraGemmError):
+        lg.set_kernel_variant(3)
