@@ -131,8 +131,12 @@ __device__ __forceinline__ void record_timeout(volatile int* abort_flag) {
 __device__ __noinline__ bool wait_slow(uint32_t bar, uint32_t parity, uint64_t limit_ns, volatile int* abort_flag,
                                        bool cluster_scope) {
   const uint64_t t0 = globaltimer_ns();
+  // Sleep in slices of at most 20 us (woken early when the phase completes),
+  // never past the wait's own limit.
+  const uint32_t hint = (uint32_t)(limit_ns < 20000ull ? limit_ns : 20000ull);
   for (;;) {
-    if (cluster_scope ? mbar_try_wait_cluster(bar, parity) : mbar_try_wait(bar, parity)) return true;
+    if (cluster_scope ? mbar_try_wait_cluster_sleep(bar, parity, hint) : mbar_try_wait_sleep(bar, parity, hint))
+      return true;
     if (*abort_flag) return false;
     if (globaltimer_ns() - t0 >= limit_ns) {
       record_timeout(abort_flag);
