@@ -45,15 +45,95 @@ __device__ __forceinline__ Words4 philox4x32_10(uint64_t block, uint32_t k0, uin
 
 // Box-Muller (Box and Muller, Ann. Math. Statist. 29, 1958) on one pair of
 // words: u1 = ((a >> 8) + 1) 2^-24 in (0, 1], u2 = (b >> 8) 2^-24 in [0, 1);
-// returns rho cos(2 pi u2) and rho sin(2 pi u2) with rho = sqrt(-2 ln u1).
-// Evaluated in double so that the FP32 result is rounded once from a value
-// accurate to far better than half an FP32 ulp.
-__device__ __forceinline__ void box_muller(uint32_t a, uint32_t b, double& e_cos, double& e_sin) {
-  const double u1 = (double)((a >> 8) + 1u) * 0x1p-24;
-  const double u2 = (double)(b >> 8) * 0x1p-24;
-  const double rho = sqrt(-2.0 * log(u1));
+// returns rho cos(2 pi u2) and rho sin(2 pi u2) with rho = sqrt(-2 ln u1), in
+// double and within a few double ulps of the exact values, so that the FP32
+// results (and any blend computed from them in double) round as the exact
+// values would.  Both uniforms are 24-bit integers scaled by 2^-24, which lets
+// every range reduction below be exact integer work; the two constant tables
+// come from gen_bm_tables.py and are staged in shared memory by the caller.
+// ---------------------------------------------------------------------------
+struct BmLogEntry {
+  double inv_c;  // 1 / c_i cut to 28 significant bits, c_i = 1 + i / 256
+  double L;      // -ln(inv_c), or -ln(2 inv_c) for i > LG_BM_LOG_SWITCH
+};
+struct BmTrigEntry {
+  double s, c;  // sin, cos of 2 pi i / 256 (exact 0 and +-1 at quarter turns)
+};
+struct BmTables {
+  const BmLogEntry* log;   // 257 entries
+  const BmTrigEntry* trig; // 256 entries
+};
+constexpr int kBmLogSwitch = 106;
+
+__device__ __forceinline__ double bits_to_double(uint64_t b) { return __longlong_as_double((long long)b); }
+
+// ln(n 2^-24) for an integer n in [1, 2^24] (Tang's table method).  With
+// n = m 2^kf, m in [1, 2), the nearest grid point c_i = 1 + i/256 gives
+// r = m inv_c - 1 exactly (m has <= 24 significant bits, inv_c 28) and
+// |r| <= 2^-9 + 2^-27, so log1p(r) to the r^6 term is within 2^-56 |r|.
+// Past c = sqrt 2 the entry already holds ln(c/2) and the exponent is one
+// higher, so a nonzero multiple of ln 2 always dominates the table term
+// (|ln u1| >= ln 2 - 0.35) and no step cancels.
+__device__ __forceinline__ double ln_grid24(uint32_t n, const BmLogEntry* tab) {
+  const int kf = 31 - __clz(n);
+  const uint32_t top = n << (31 - kf);                      // leading one at bit 31
+  const int i = (int)(((top >> 22) + 1u) >> 1) - 256;       // 0..256
+  const BmLogEntry e = tab[i];
+  const int j = 24 - kf - (i > kBmLogSwitch ? 1 : 0);        // 0..24
+  // m = n 2^-kf assembled from the bits of n (exact)
+  const double m = bits_to_double(((uint64_t)n << (52 - kf)) + ((uint64_t)1022 << 52));
+  const double r = fma(m, e.inv_c, -1.0);
+  double p = -1.0 / 6.0;
+  p = fma(p, r, 1.0 / 5.0);
+  p = fma(p, r, -1.0 / 4.0);
+  p = fma(p, r, 1.0 / 3.0);
+  p = fma(p, r, -0.5);
+  const double log1p_r = fma(r * r, p, r);
+  // (double)j from the bits of 2^52 + j
+  const double jd = bits_to_double(0x4330000000000000ull + (uint64_t)j) - 0x1p52;
+  return fma(-jd, 0.6931471805599453094, e.L + log1p_r);
+}
+
+// sqrt(y) for y = +-0 or y in [2^-24, 64): an FP32 reciprocal square root
+// seed, one Newton step on 1/sqrt(y) in double (relative error ~2^-44), then
+// one correction of y / sqrt(y) (error ~2^-88 before the final rounding).
+__device__ __forceinline__ double sqrt_seeded(double y) {
+  const uint32_t hi = max((uint32_t)__double2hiint(y) & 0x7FFFFFFFu, 0x3E700000u);  // finite seed at y = +-0
+  const float yf = __uint_as_float((hi - (896u << 20)) << 3);        // y truncated to FP32
+  float rf;
+  asm("rsqrt.approx.ftz.f32 %0, %1;" : "=f"(rf) : "f"(yf));
+  double r = bits_to_double(((uint64_t)__float_as_uint(rf) << 29) + ((uint64_t)896 << 52));
+  const double t = y * r;
+  r = fma(0.5 * r, fma(-t, r, 1.0), r);
+  const double s0 = y * r;
+  return fma(fma(-s0, s0, y), 0.5 * r, s0);
+}
+
+// sin and cos of 2 pi b 2^-24 for an integer b in [0, 2^24): the nearest
+// 1/256 turn comes from the table, the remainder theta (|theta| <= pi/256,
+// exact integer times 2 pi 2^-24) from short Maclaurin series (truncation
+// below 1e-20 relative), combined by the angle-addition formulas.  Near a
+// zero of sin or cos the table term is exactly zero, so the result keeps full
+// relative accuracy.
+__device__ __forceinline__ void sincos_turn24(uint32_t b, const BmTrigEntry* tab, double& s, double& c) {
+  const uint32_t iu = ((b >> 15) + 1u) >> 1;                 // nearest multiple of 2^16, 0..256
+  const int32_t ri = (int32_t)b - (int32_t)(iu << 16);       // -2^15 .. 2^15 - 1
+  const BmTrigEntry t = tab[iu & 255u];
+  // (double)ri from the bits of 1.5 2^52 + ri
+  const double rd = bits_to_double(0x4338000000000000ull + (uint64_t)(int64_t)ri) - 0x1.8p52;
+  const double th = rd * (6.283185307179586 * 0x1p-24);
+  const double z = th * th;
+  const double sth = fma(th * z, fma(z, fma(z, -1.0 / 5040.0, 1.0 / 120.0), -1.0 / 6.0), th);
+  const double cm1 = z * fma(z, fma(z, -1.0 / 720.0, 1.0 / 24.0), -0.5);  // cos(theta) - 1
+  s = fma(t.s, cm1, fma(t.c, sth, t.s));
+  c = fma(t.c, cm1, fma(-t.s, sth, t.c));
+}
+
+__device__ __forceinline__ void box_muller(uint32_t a, uint32_t b, const BmTables& tab, double& e_cos,
+                                           double& e_sin) {
+  const double rho = sqrt_seeded(-2.0 * ln_grid24((a >> 8) + 1u, tab.log));
   double s, c;
-  sincospi(2.0 * u2, &s, &c);
+  sincos_turn24(b >> 8, tab.trig, s, c);
   e_cos = rho * c;
   e_sin = rho * s;
 }

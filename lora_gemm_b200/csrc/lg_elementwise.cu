@@ -10,6 +10,7 @@
 // 精修方案", section "三个步如何完成工作".
 #include <algorithm>
 
+#include "lg_bm_tables.inc"
 #include "lg_device.cuh"
 #include "lg_internal.h"
 
@@ -18,6 +19,19 @@ namespace lg {
 namespace {
 
 constexpr int kThreads = 256;
+
+static_assert(LG_BM_LOG_SWITCH == kBmLogSwitch, "log table built for another switch point");
+__device__ const BmLogEntry g_bm_log[LG_BM_LOG_ENTRIES] = LG_BM_LOG_TABLE;
+__device__ const BmTrigEntry g_bm_trig[LG_BM_TRIG_ENTRIES] = LG_BM_TRIG_TABLE;
+
+// Copies the Box-Muller tables (8 KB) into the block's shared memory, where
+// the data-dependent lookups cost one shared load each.
+__device__ __forceinline__ BmTables stage_bm_tables(BmLogEntry* s_log, BmTrigEntry* s_trig) {
+  for (int i = threadIdx.x; i < LG_BM_LOG_ENTRIES; i += blockDim.x) s_log[i] = g_bm_log[i];
+  for (int i = threadIdx.x; i < LG_BM_TRIG_ENTRIES; i += blockDim.x) s_trig[i] = g_bm_trig[i];
+  __syncthreads();
+  return BmTables{s_log, s_trig};
+}
 
 __device__ __forceinline__ int64_t gtid() { return (int64_t)blockIdx.x * blockDim.x + threadIdx.x; }
 __device__ __forceinline__ int64_t gstride() { return (int64_t)gridDim.x * blockDim.x; }
@@ -31,18 +45,22 @@ __global__ void __launch_bounds__(kThreads) k_philox_u32(uint4* __restrict__ out
 }
 
 // The four normals of Philox block `block`.
-__device__ __forceinline__ void normals4(uint64_t block, uint32_t k0, uint32_t k1, double (&e)[4]) {
+__device__ __forceinline__ void normals4(uint64_t block, uint32_t k0, uint32_t k1, const BmTables& tab,
+                                         double (&e)[4]) {
   const Words4 r = philox4x32_10(block, k0, k1);
-  box_muller(r.w0, r.w1, e[0], e[1]);
-  box_muller(r.w2, r.w3, e[2], e[3]);
+  box_muller(r.w0, r.w1, tab, e[0], e[1]);
+  box_muller(r.w2, r.w3, tab, e[2], e[3]);
 }
 
-__global__ void __launch_bounds__(kThreads) k_philox_normal(float* __restrict__ eps, int64_t n, uint32_t k0,
+__global__ void __launch_bounds__(kThreads, 8) k_philox_normal(float* __restrict__ eps, int64_t n, uint32_t k0,
                                                             uint32_t k1, uint64_t block0) {
+  __shared__ BmLogEntry s_log[LG_BM_LOG_ENTRIES];
+  __shared__ BmTrigEntry s_trig[LG_BM_TRIG_ENTRIES];
+  const BmTables tab = stage_bm_tables(s_log, s_trig);
   const int64_t n_blocks = (n + 3) / 4;
   for (int64_t b = gtid(); b < n_blocks; b += gstride()) {
     double e[4];
-    normals4(block0 + (uint64_t)b, k0, k1, e);
+    normals4(block0 + (uint64_t)b, k0, k1, tab, e);
     if (4 * b + 4 <= n) {
       reinterpret_cast<float4*>(eps)[b] = make_float4((float)e[0], (float)e[1], (float)e[2], (float)e[3]);
     } else {
@@ -54,13 +72,16 @@ __global__ void __launch_bounds__(kThreads) k_philox_normal(float* __restrict__ 
 // x = (1 - sigma) up + sigma eps, blended in double from the unrounded eps
 // and rounded once to FP32.  x may alias up (each element is read before it
 // is written by the same thread), so neither pointer is restrict.
-__global__ void __launch_bounds__(kThreads) k_renoise(const float* up, float* x, int64_t n,
+__global__ void __launch_bounds__(kThreads, 8) k_renoise(const float* up, float* x, int64_t n,
                                                       double sigma, uint32_t k0, uint32_t k1, uint64_t block0) {
+  __shared__ BmLogEntry s_log[LG_BM_LOG_ENTRIES];
+  __shared__ BmTrigEntry s_trig[LG_BM_TRIG_ENTRIES];
+  const BmTables tab = stage_bm_tables(s_log, s_trig);
   const double keep = 1.0 - sigma;
   const int64_t n_blocks = (n + 3) / 4;
   for (int64_t b = gtid(); b < n_blocks; b += gstride()) {
     double e[4];
-    normals4(block0 + (uint64_t)b, k0, k1, e);
+    normals4(block0 + (uint64_t)b, k0, k1, tab, e);
     if (4 * b + 4 <= n) {
       const float4 u = __ldcs(reinterpret_cast<const float4*>(up) + b);
       float4 o;

@@ -1,0 +1,99 @@
+"""Host checks of the constant tables behind the device Box-Muller transform.
+
+The committed include must be exactly what its generator writes, and the
+properties the device code relies on must hold: every 1/c_i has at most 28
+significant bits (so m * inv_c is exact for a 24-bit mantissa m), it is
+within 2^-27 of 1/c_i, the log entries are the logarithms they stand for,
+the trig entries are exact at quarter turns and on the unit circle.  Pure
+host work: no GPU, no oracle.
+"""
+
+import importlib.util
+import math
+import os
+import random
+import struct
+from fractions import Fraction
+
+import pytest
+
+CSRC = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "lora_gemm_b200", "csrc")
+
+
+def _load_gen():
+    spec = importlib.util.spec_from_file_location("gen_bm_tables", os.path.join(CSRC, "gen_bm_tables.py"))
+    mod = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(mod)
+    return mod
+
+
+gen = _load_gen()
+
+
+def _mantissa_bits_used(x):
+    b = struct.unpack("<Q", struct.pack("<d", x))[0] & ((1 << 52) - 1)
+    if b == 0:
+        return 1
+    tz = (b & -b).bit_length() - 1
+    return 53 - tz
+
+
+def test_committed_include_matches_generator():
+    with open(os.path.join(CSRC, "lg_bm_tables.inc")) as f:
+        assert f.read() == gen.render()
+
+
+def test_log_table_invariants():
+    rows = gen.log_table()
+    assert len(rows) == 257
+    for i, (inv, L) in enumerate(rows):
+        c = 1.0 + i / 256.0
+        assert _mantissa_bits_used(inv) <= 28
+        assert abs(c * inv - 1.0) <= 2.0**-27
+        want = -math.log(2.0 * inv) if i > gen.LOG_SWITCH else -math.log(inv)
+        assert L == want
+        # the stored term never exceeds half of ln 2, so a nonzero multiple of
+        # ln 2 always dominates it
+        assert abs(L) <= 0.35
+    assert rows[0] == (1.0, 0.0) and rows[256] == (0.5, 0.0)
+    # the switch sits at sqrt(2): the entries on either side straddle it
+    assert 1 + gen.LOG_SWITCH / 256 < math.sqrt(2) < 1 + (gen.LOG_SWITCH + 1) / 256
+
+
+def test_log_reduction_is_exact_for_every_mantissa_class():
+    """r = m inv_c - 1 is a double exactly (so one fused multiply-add returns
+    it unrounded) for 24-bit mantissas m in every table class, including the
+    class edges, and |r| stays within 2^-9 + 2^-27."""
+    rows = gen.log_table()
+    rng = random.Random(0)
+    for i in range(257):
+        lo = max(1.0, 1.0 + (i - 0.5) / 256.0)
+        hi = min(2.0, 1.0 + (i + 0.5) / 256.0)
+        ks = [math.ceil(lo * 2**23), math.ceil(hi * 2**23) - 1] + [rng.randrange(math.ceil(lo * 2**23), math.ceil(hi * 2**23)) for _ in range(20)]
+        for k in ks:
+            m = Fraction(k, 2**23)  # m in [1, 2) with 24 significant bits
+            r = m * Fraction(rows[i][0]) - 1
+            assert Fraction(float(r)) == r
+            assert abs(r) <= Fraction(1, 512) + Fraction(1, 2**27)
+
+
+def test_trig_table_invariants():
+    rows = gen.trig_table()
+    assert len(rows) == 256
+    exact = {0: (0.0, 1.0), 64: (1.0, 0.0), 128: (0.0, -1.0), 192: (-1.0, 0.0)}
+    for i, (s, c) in enumerate(rows):
+        if i in exact:
+            assert (s, c) == exact[i]
+            assert math.copysign(1.0, s) > 0 or s != 0.0  # no negative zeros
+            assert math.copysign(1.0, c) > 0 or c != 0.0
+        assert abs(s * s + c * c - 1.0) <= 4e-16
+        a = 2 * math.pi * i / 256
+        assert abs(s - math.sin(a)) <= 1e-15 and abs(c - math.cos(a)) <= 1e-15
+
+
+@pytest.mark.parametrize("i", [1, 37, 64 + 5, 128 + 63, 255])
+def test_trig_table_symmetry(i):
+    rows = gen.trig_table()
+    s, c = rows[i]
+    s2, c2 = rows[(i + 64) % 256]  # a quarter turn later: (c, -s)
+    assert (s2, c2) == (c + 0.0, -s + 0.0)
