@@ -64,42 +64,21 @@ def load_peaks():
 
 
 # ---------------------------------------------------------------------------
-# Distributed plumbing (one process per GPU; NCCL only for barrier / max).
+# Distributed plumbing: lora_gemm_b200.dist (one process per GPU; NCCL only
+# for the barrier and the max over ranks).
 # ---------------------------------------------------------------------------
-def dist_setup(n_gpus):
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
-    if world != n_gpus:
-        raise SystemExit(f"--gpus {n_gpus} but WORLD_SIZE={world}")
-    if world > 1:
-        import datetime
+def _dist():
+    from lora_gemm_b200 import dist
 
-        import torch.distributed as dist
-
-        torch.cuda.set_device(local)
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=600),
-                                device_id=torch.device("cuda", local))
-    else:
-        torch.cuda.set_device(0)
-    return rank, world, local
+    return dist
 
 
 def barrier(world):
-    if world > 1:
-        import torch.distributed as dist
-
-        dist.barrier()
+    _dist().barrier(world)
 
 
 def max_over_ranks(value, world):
-    if world == 1:
-        return value
-    import torch.distributed as dist
-
-    t = torch.tensor([value], dtype=torch.float64, device="cuda")
-    dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    return float(t.item())
+    return _dist().max_over_ranks(value, world)
 
 
 # ---------------------------------------------------------------------------
@@ -183,7 +162,7 @@ def layer_flops(M, K, N, R):
 class Problem:
     """Device-resident inputs and outputs of one 2K step."""
 
-    def __init__(self, w, dev, tokens=None):
+    def __init__(self, w, dev, tokens=None, noise_offset=0):
         from lora_gemm_b200 import synth
         import lora_gemm_b200 as lg
 
@@ -210,6 +189,7 @@ class Problem:
         self.x_lat = torch.empty_like(self.up)
         self.v = [synth.velocity(w, k, dev) for k in range(3)]
         self.sigmas = [float(torch.tensor(s, dtype=torch.float32)) for s in synth.SIGMA_SCHEDULE]
+        self.noise_offset = noise_offset  # this rank's slice of the Philox stream
         self.scales = synth.ADAPTER_SCALES
 
 
@@ -230,7 +210,7 @@ def run_step(P, ev=None):
 
     for L in P.layers:
         rec("lora_merge", lambda L=L: lg.lora_merge(L["As"], L["Bs"], P.scales, L["A_cat"], L["B_cat"]))
-    rec("renoise", lambda: lg.renoise(P.up, P.sigmas[0], P.w.seed, out=P.x_lat))
+    rec("renoise", lambda: lg.renoise(P.up, P.sigmas[0], P.w.seed, offset=P.noise_offset, out=P.x_lat))
     for k, L in enumerate(P.layers):
         rec(f"lora_linear{k}", lambda L=L: lg.lora_linear(L["x"], L["W"], L["A_cat"], L["B_cat"], y=L["y"],
                                                           workspace=L["ws"]))
@@ -254,7 +234,7 @@ def run_ours(args, rank, world, local):
     peaks = load_peaks()
     dev = torch.device("cuda", torch.cuda.current_device())
     w = synth.WORKLOADS[args.workload]
-    P = Problem(w, dev, tokens=args.tokens)
+    P = Problem(w, dev, tokens=args.tokens, noise_offset=_dist().noise_offset(rank, w.latent_numel))
     torch.cuda.synchronize()
 
     for _ in range(args.warmup):
@@ -290,7 +270,7 @@ def run_ours(args, rank, world, local):
     for name, s, e in ev:
         per.setdefault(name, []).append(s.elapsed_time(e))
     M = P.M
-    value = world * M * args.steps / (elapsed_ms * 1e-3)
+    value = _dist().whole_job_rate(M, world, args.steps, elapsed_ms)
 
     # Dominant kernel: lora_linear (tensor-bound).
     flops = [layer_flops(M, L["K"], L["N"], P.R) for L in P.layers]
@@ -437,7 +417,7 @@ def run_e2e(P, args, world):
     torch.cuda.synchronize()
     barrier(world)
     ms = max_over_ranks(s.elapsed_time(e), world)
-    return {"value": round(world * P.M * steps / (ms * 1e-3), 1), "unit": UNIT,
+    return {"value": round(_dist().whole_job_rate(P.M, world, steps, ms), 1), "unit": UNIT,
             "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h), "steps": steps,
             "ms_per_step": round(ms / steps, 3)}
 
@@ -579,16 +559,13 @@ def main():
         print(json.dumps(run_reference(args, rank, world)), flush=True)
         return
 
-    rank, world, local = dist_setup(args.gpus)
+    rank, world, local = _dist().init(args.gpus, backend="nccl")
     try:
         result = run_ours(args, rank, world, local)
         if rank == 0:
             print(json.dumps(result), flush=True)
     finally:
-        if world > 1:
-            import torch.distributed as dist
-
-            dist.destroy_process_group()
+        _dist().destroy(world)
 
 
 if __name__ == "__main__":
