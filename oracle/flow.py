@@ -13,7 +13,19 @@ Few-Step Diffusion" (agientry.com, English article).
 
 Page "Open-H3-Regenerate-2K-IC" (wujieai.com), section
 "三步接着放大的草稿画，八步从噪声重画": the IC variant starts from
-sigma = 0.835 (up3) or 0.923 (up4) with the same blend.
+sigma = 0.835 (up3) or 0.923 (up4) with the same blend, or from pure noise
+(sigma = 1, hf8); all three routes share HyperFlow's eight-step noise table
+with video shift 12; up3 then takes the last three steps of that table, up4
+one step more, hf8 all eight; the reference row is blended with 0.1 % noise
+(sigma = 0.001).
+
+Reading of the table (the page names it but prints no formula): "video
+shift 12" is the flow-matching time shift sigma = s t / (1 + (s - 1) t) on
+the uniform grid t_k = 1 - k/8, k = 0..8.  At t = 1/2 it gives 12/13 =
+0.923..., the printed up4 start.  A route starts at its printed sigma0 and
+then visits every table point strictly below it, which yields three steps
+for up3 (0.835 -> 0.8 -> 0.632 -> 0), four for up4 and eight for hf8, as the
+page counts them.
 
 Reading of the decimals (the pages print decimals only): each sigma is the
 FP32 value nearest to the printed decimal, and both the kernels and this
@@ -27,6 +39,12 @@ import numpy as np
 SCHEDULE_DECIMAL = (0.909, 0.857, 0.667, 0.0)
 # IC starts, "三步接着放大的草稿画，八步从噪声重画".
 IC_STARTS_DECIMAL = (0.835, 0.923)
+# Same section: the shared eight-step table, its video shift, the three
+# routes' printed starts and the reference row's noise share.
+HYPERFLOW_STEPS = 8
+HYPERFLOW_SHIFT = 12.0
+IC_ROUTES_DECIMAL = {"up3": 0.835, "up4": 0.923, "hf8": 1.0}
+REFERENCE_ROW_SIGMA_DECIMAL = 0.001
 
 
 def as_fp32(value):
@@ -75,3 +93,21 @@ def refine(up, eps, schedule, velocity):
         z = euler_step(z, velocity(z, k), schedule[k], schedule[k + 1])
         out.append(z)
     return out
+
+
+def shifted_sigma(t, shift):
+    """Time shift of the flow-matching grid: sigma = s t / (1 + (s - 1) t), FP64."""
+    t = float(t)
+    return shift * t / (1.0 + (shift - 1.0) * t)
+
+
+def hyperflow_table(n_steps=HYPERFLOW_STEPS, shift=HYPERFLOW_SHIFT):
+    """sigma at t_k = 1 - k / n_steps for k = 0..n_steps (FP64, from 1 down to 0)."""
+    return [shifted_sigma(1.0 - k / n_steps, shift) for k in range(n_steps + 1)]
+
+
+def ic_ladder(sigma0_decimal, n_steps=HYPERFLOW_STEPS, shift=HYPERFLOW_SHIFT):
+    """The sigmas a route visits: its printed start, then every table point
+    strictly below it; each the exact FP32 value (see as_fp32)."""
+    start = as_fp32(sigma0_decimal)
+    return [start] + [as_fp32(s) for s in hyperflow_table(n_steps, shift) if as_fp32(s) < start]

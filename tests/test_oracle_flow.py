@@ -87,3 +87,72 @@ def test_euler_special_cases():
     np.testing.assert_array_equal(flow.euler_step(x, v, 0.5, 0.5), x)
     # Stepping to sigma' = sigma - 1 adds v with a minus sign.
     np.testing.assert_allclose(flow.euler_step(x, v, 1.0, 0.0), x - v, rtol=0, atol=1e-15)
+
+
+# --- HyperFlow table and the IC routes ("三步接着放大的草稿画，八步从噪声重画") ---
+
+
+def test_hyperflow_constants_match_page():
+    g = _golden("schedule.json")["hyperflow"]
+    assert flow.HYPERFLOW_STEPS == g["steps"] and flow.HYPERFLOW_SHIFT == g["video_shift"]
+    assert {r: v["sigma0"] for r, v in g["routes"].items()} == flow.IC_ROUTES_DECIMAL
+    assert flow.REFERENCE_ROW_SIGMA_DECIMAL == g["reference_row_sigma"]
+
+
+@pytest.mark.parametrize("route", ["up3", "up4", "hf8"])
+def test_route_step_counts_match_page(route):
+    """The page counts three steps for up3, one more for up4 and eight for hf8."""
+    g = _golden("schedule.json")["hyperflow"]["routes"][route]
+    lad = flow.ic_ladder(g["sigma0"])
+    assert len(lad) - 1 == g["steps"]
+    assert lad[0] == flow.as_fp32(g["sigma0"]) and lad[-1] == 0.0
+    assert all(a > b for a, b in zip(lad, lad[1:]))
+
+
+def test_hyperflow_table_properties():
+    tab = flow.hyperflow_table()
+    assert len(tab) == 9 and tab[0] == 1.0 and tab[-1] == 0.0  # hf8 starts from pure noise
+    # the printed up4 start is the table point at t = 1/2, to the printed digits
+    assert round(tab[4], 3) == 0.923
+    # inverting the shift, t = sigma / (s - (s - 1) sigma), gives back the uniform grid
+    s = flow.HYPERFLOW_SHIFT
+    for k, sig in enumerate(tab):
+        assert abs(sig / (s - (s - 1) * sig) - (1 - k / 8)) < 1e-15
+    # shift 1 is the unshifted grid; a larger shift pushes every interior point up
+    assert flow.hyperflow_table(shift=1.0) == [1 - k / 8 for k in range(9)]
+    for a, b in zip(flow.hyperflow_table(shift=3.0)[1:-1], tab[1:-1]):
+        assert a < b
+
+
+def test_route_coefficients_exact_in_fp32():
+    """Sterbenz again: every dt of every route and 1 - sigma0 (sigma0 >= 1/2)
+    are exact in FP32, so the kernels' coefficients equal the oracle's."""
+    for start in flow.IC_ROUTES_DECIMAL.values():
+        lad = [np.float32(x) for x in flow.ic_ladder(start)]
+        assert float(np.float32(1.0) - lad[0]) == 1.0 - float(lad[0])
+        for a, b in zip(lad[:-1], lad[1:]):
+            assert float(b - a) == float(b) - float(a)
+
+
+@pytest.mark.parametrize("route", ["up3", "up4", "hf8"])
+def test_routes_recover_z0_with_exact_velocity(route):
+    rng = np.random.default_rng(7)
+    z0 = rng.standard_normal(5000)
+    eps = rng.standard_normal(5000)
+    lad = flow.ic_ladder(flow.IC_ROUTES_DECIMAL[route])
+    zs = flow.refine(z0, eps, lad, lambda z, k: flow.exact_velocity(z0, eps))
+    for z, sig in zip(zs, lad):
+        np.testing.assert_allclose(z, flow.flow_point(z0, eps, sig), rtol=0, atol=1e-14)
+    if route == "hf8":
+        assert np.array_equal(zs[0], eps)  # sigma 1: the draft does not enter the start
+    assert np.abs(zs[-1] - z0).max() < 1e-14
+
+
+def test_reference_row_blend():
+    """99.9 % draft, 0.1 % noise: the FP32 sigma is within 2^-34 of 0.001 and
+    the blend is the exact convex combination."""
+    sig = flow.as_fp32(flow.REFERENCE_ROW_SIGMA_DECIMAL)
+    assert abs(sig - 0.001) < 2.0**-34
+    up = np.array([1.0, -2.0, 0.0])
+    eps = np.array([0.0, 1.0, 5.0])
+    np.testing.assert_array_equal(flow.renoise(up, eps, sig), (1 - sig) * up + sig * eps)
