@@ -224,6 +224,32 @@ lg_status lg_euler_step(float* x, const float* v, int64_t n, float sigma, float 
                         void* stream);
 
 /* ------------------------------------------------------------------------
+ * lg_shift_ladder -- the sigmas a sampling route visits on a time-shifted
+ * flow-matching table.  Host computation only (no device work, no stream):
+ *
+ *   table_k = shift t_k / (1 + (shift - 1) t_k),  t_k = 1 - k / n_steps,
+ *             k = 0..n_steps (1 down to 0), evaluated in double and rounded
+ *             to FP32;
+ *   ladder  = sigma0, then every table value strictly below sigma0.
+ *
+ * Page "Open-H3-Regenerate-2K-IC", section "三步接着放大的草稿画，八步从噪声重画":
+ * the up3, up4 and hf8 routes share HyperFlow's eight-step table with video
+ * shift 12; they start at 0.835, 0.923 and 1 and take 3, 4 and 8 steps.  The
+ * page prints no formula; the time shift above is this library's reading of
+ * "video shift 12" (it puts the table point at t = 1/2 at 12/13 = 0.923...).
+ * The route is then: lg_renoise at ladder[0], lg_euler_step from ladder[k] to
+ * ladder[k + 1] for each k.
+ *
+ *   sigma0   0 < sigma0 <= 1.
+ *   n_steps  1 .. 4096.   shift  finite, > 0.
+ *   out      HOST FP32 array with room for `cap` values; the ladder has at
+ *            most n_steps + 1 values.  *len receives the count.
+ *   Returns LG_ERR_INVALID_ARG (writing nothing) for an argument out of range,
+ *   null pointers, or cap smaller than the ladder.
+ * ---------------------------------------------------------------------- */
+lg_status lg_shift_ladder(float sigma0, int n_steps, double shift, float* out, int cap, int* len);
+
+/* ------------------------------------------------------------------------
  * Generator hooks (same generator as lg_renoise), for testing.
  *
  * lg_philox_u32: out[4b + t] = word t of Philox4x32-10(counter of block

@@ -59,6 +59,11 @@ _SIGNATURES = {
     "lg_euler_step": (
         ctypes.c_int, [_c_void_p, _c_void_p, ctypes.c_int64, ctypes.c_float, ctypes.c_float, _c_void_p]
     ),
+    "lg_shift_ladder": (
+        ctypes.c_int,
+        [ctypes.c_float, ctypes.c_int, ctypes.c_double, ctypes.POINTER(ctypes.c_float), ctypes.c_int,
+         ctypes.POINTER(ctypes.c_int)],
+    ),
     "lg_philox_u32": (ctypes.c_int, [_c_void_p, ctypes.c_int64, ctypes.c_uint64, ctypes.c_uint64, _c_void_p]),
     "lg_philox_normal": (ctypes.c_int, [_c_void_p, ctypes.c_int64, ctypes.c_uint64, ctypes.c_uint64, _c_void_p]),
 }
@@ -263,6 +268,22 @@ def euler_step(x, v, sigma, sigma_next):
         st = lib.lg_euler_step(_ptr(x), _ptr(v), x.numel(), float(sigma), float(sigma_next), _stream(x.device))
     _check(st, "lg_euler_step")
     return x
+
+
+# Routes of the IC sampler: printed start sigma on HyperFlow's eight-step,
+# shift-12 table (page "Open-H3-Regenerate-2K-IC", section
+# "三步接着放大的草稿画，八步从噪声重画").
+IC_ROUTES = {"up3": 0.835, "up4": 0.923, "hf8": 1.0}
+
+
+def shift_ladder(sigma0, n_steps=8, shift=12.0):
+    """The FP32 sigmas a route visits: sigma0, then every point of the
+    shift-`shift`, `n_steps`-step table below it (host computation)."""
+    buf = (ctypes.c_float * (int(n_steps) + 2))()
+    n = ctypes.c_int(0)
+    st = lib.lg_shift_ladder(float(sigma0), int(n_steps), float(shift), buf, len(buf), ctypes.byref(n))
+    _check(st, "lg_shift_ladder")
+    return [float(buf[i]) for i in range(n.value)]
 
 
 def philox_u32(n_blocks, seed, block_offset=0, out=None, device=None):

@@ -246,6 +246,27 @@ lg_status lg_euler_step(float* x, const float* v, int64_t n, float sigma, float 
   return launched(lg::launch_euler(x, v, n, dt, sms, as_stream(stream)), 1);
 }
 
+lg_status lg_shift_ladder(float sigma0, int n_steps, double shift, float* out, int cap, int* len) {
+  if (!out || !len || !(sigma0 > 0.0f && sigma0 <= 1.0f) || n_steps < 1 || n_steps > 4096 ||
+      !std::isfinite(shift) || !(shift > 0.0)) {
+    return LG_ERR_INVALID_ARG;
+  }
+  float ladder[4097 + 1];
+  int count = 0;
+  ladder[count++] = sigma0;
+  for (int k = 0; k <= n_steps; ++k) {
+    const double t = 1.0 - (double)k / (double)n_steps;
+    const double num = shift * t;
+    const double den = 1.0 + (shift - 1.0) * t;
+    const float sig = (float)(num / den);
+    if (sig < sigma0) ladder[count++] = sig;
+  }
+  if (cap < count) return LG_ERR_INVALID_ARG;
+  for (int i = 0; i < count; ++i) out[i] = ladder[i];
+  *len = count;
+  return LG_OK;
+}
+
 lg_status lg_philox_u32(uint32_t* out, int64_t n_blocks, uint64_t seed, uint64_t block_offset, void* stream) {
   if (n_blocks < 0) return LG_ERR_INVALID_ARG;
   if (n_blocks == 0) return LG_OK;
