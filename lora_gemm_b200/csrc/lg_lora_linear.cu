@@ -216,6 +216,16 @@ __device__ void run_producer(const CUtensorMap* tm_x, const CUtensorMap* tm_w, c
       tma_load_2d(dst, m, full0 + 8 * stage, c0, c1);
     }
   };
+  // x panels are re-read once per N tile: keep them in L2 ahead of the
+  // streamed weight tiles.
+  const uint64_t pol_x = l2_policy_evict_last();
+  auto load_x = [&](uint32_t dst, int c0, int c1) {
+    if constexpr (PAIR) {
+      tma_load_2d_pair_hint(dst, tm_x, full0 + 8 * stage, c0, c1, pol_x);
+    } else {
+      tma_load_2d_hint(dst, tm_x, full0 + 8 * stage, c0, c1, pol_x);
+    }
+  };
   for (int p = (int)cid; ok && p < a.num_panels; p += (int)ncl, ++it) {
     const int m0 = p * C::PANEL + half * BM;
     for (int j = 0; ok && j < a.n_chunks; ++j, ++sweep) {
@@ -229,7 +239,7 @@ __device__ void run_producer(const CUtensorMap* tm_x, const CUtensorMap* tm_w, c
         }
         const uint32_t sa = smem_base + stage * C::STAGE;
         if (posts_tx) mbar_arrive_expect_tx(full_local + 8 * stage, tx_a);
-        load(tm_x, sa, kb * BK, m0);
+        load_x(sa, kb * BK, m0);
         load(tm_a, sa + A_BYTES, kb * BK, first + half * (int)a_rows);
         ++fills;
         advance(stage, phase, stages);
@@ -252,7 +262,7 @@ __device__ void run_producer(const CUtensorMap* tm_x, const CUtensorMap* tm_w, c
         }
         const uint32_t sa = smem_base + stage * C::STAGE;
         if (posts_tx) mbar_arrive_expect_tx(full_local + 8 * stage, tx_k);
-        load(tm_x, sa, kb * BK, m0);
+        load_x(sa, kb * BK, m0);
         load(tm_w, sa + A_BYTES, kb * BK, n0);
         ++fills;
         advance(stage, phase, stages);
@@ -485,6 +495,8 @@ __device__ void run_epilogue(const Args& a, Control* ctl, uint32_t smem_base, ui
   uint32_t acc_phase = 0;
   uint32_t it = 0;
   bool ok = true;
+  // y is written once and not read here: let it leave L2 first.
+  const uint64_t pol_y = l2_policy_evict_first();
   auto release_acc = [&]() {
     tc_fence_before();
     __syncwarp();
@@ -560,11 +572,10 @@ __device__ void run_epilogue(const Args& a, Control* ctl, uint32_t smem_base, ui
         auto store8 = [&](int g, const uint32_t* v) {
           const int col = col0 + 8 * g;
           if (col < a.N) {
-            *reinterpret_cast<uint4*>(dst_row + col) =
-                make_uint4(pack_bf16x2(__uint_as_float(v[0]), __uint_as_float(v[1])),
-                           pack_bf16x2(__uint_as_float(v[2]), __uint_as_float(v[3])),
-                           pack_bf16x2(__uint_as_float(v[4]), __uint_as_float(v[5])),
-                           pack_bf16x2(__uint_as_float(v[6]), __uint_as_float(v[7])));
+            st_global_v4_hint(dst_row + col, pack_bf16x2(__uint_as_float(v[0]), __uint_as_float(v[1])),
+                              pack_bf16x2(__uint_as_float(v[2]), __uint_as_float(v[3])),
+                              pack_bf16x2(__uint_as_float(v[4]), __uint_as_float(v[5])),
+                              pack_bf16x2(__uint_as_float(v[6]), __uint_as_float(v[7])), pol_y);
           }
         };
 #pragma unroll
