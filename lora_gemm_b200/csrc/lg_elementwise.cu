@@ -107,31 +107,30 @@ __global__ void __launch_bounds__(kThreads) k_euler(float* __restrict__ x, const
   float4* x4 = reinterpret_cast<float4*>(x);
   const float4* v4 = reinterpret_cast<const float4*>(v);
   const int64_t stride = gstride();
-  int64_t i = gtid();
-  for (; i + (kEulerUnroll - 1) * stride < n4; i += kEulerUnroll * stride) {
+  // Every pass issues all of its loads before any arithmetic, the last
+  // (partial) pass included, so each thread keeps up to 2 x kEulerUnroll
+  // 16-byte loads in flight to the end.
+  for (int64_t i = gtid(); i < n4; i += kEulerUnroll * stride) {
     float4 a[kEulerUnroll], b[kEulerUnroll];
 #pragma unroll
     for (int u = 0; u < kEulerUnroll; ++u) {
-      a[u] = x4[i + u * stride];
-      b[u] = __ldcs(v4 + i + u * stride);
+      const int64_t j = i + u * stride;
+      if (j < n4) {
+        a[u] = x4[j];
+        b[u] = __ldcs(v4 + j);
+      }
     }
 #pragma unroll
     for (int u = 0; u < kEulerUnroll; ++u) {
-      a[u].x = fmaf(dt, b[u].x, a[u].x);
-      a[u].y = fmaf(dt, b[u].y, a[u].y);
-      a[u].z = fmaf(dt, b[u].z, a[u].z);
-      a[u].w = fmaf(dt, b[u].w, a[u].w);
-      x4[i + u * stride] = a[u];
+      const int64_t j = i + u * stride;
+      if (j < n4) {
+        a[u].x = fmaf(dt, b[u].x, a[u].x);
+        a[u].y = fmaf(dt, b[u].y, a[u].y);
+        a[u].z = fmaf(dt, b[u].z, a[u].z);
+        a[u].w = fmaf(dt, b[u].w, a[u].w);
+        x4[j] = a[u];
+      }
     }
-  }
-  for (; i < n4; i += stride) {
-    float4 a = x4[i];
-    const float4 b = __ldcs(v4 + i);
-    a.x = fmaf(dt, b.x, a.x);
-    a.y = fmaf(dt, b.y, a.y);
-    a.z = fmaf(dt, b.z, a.z);
-    a.w = fmaf(dt, b.w, a.w);
-    x4[i] = a;
   }
   if (gtid() == 0) {
     for (int64_t t = 4 * n4; t < n; ++t) x[t] = fmaf(dt, v[t], x[t]);

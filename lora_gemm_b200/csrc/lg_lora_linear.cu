@@ -876,9 +876,24 @@ cudaError_t launch_lora_linear(const LinearLaunch& p, cudaStream_t s, bool* driv
   if (e != cudaSuccess) return e;
   e = configure_kernels(dev);
   if (e != cudaSuccess) return e;
-  // Variant and cluster size (both process-wide overrides for tuning).
-  const int variant = g_variant_override ? g_variant_override : 1;
+  // Variant and cluster size (both process-wide overrides for tuning).  The
+  // automatic choice follows sustained (power-capped) sweeps on B200: private
+  // panels for small K; SM pairs, one or two per panel, for K up to 8192;
+  // single-SM pairs of CTAs beyond, where the panels' x no longer fits L2
+  // either way and the SM pairs' extra DRAM traffic costs clock.
+  int variant = g_variant_override;
   int cluster = g_cluster_override;
+  if (variant == 0) {
+    if (p.K <= 2048 || cluster == 1) {
+      variant = 1;
+      if (cluster == 0) cluster = 1;
+    } else if (p.K <= 8192) {
+      variant = 2;
+      if (cluster == 0) cluster = p.K <= 4096 ? 2 : 4;
+    } else {
+      variant = 1;
+    }
+  }
   if (variant == 1) {
     if (cluster == 0) cluster = p.K <= 2048 ? 1 : 2;
     if (cluster > 8) cluster = 8;
