@@ -55,35 +55,45 @@ namespace {
 
 constexpr int BM = 128;      // token rows per CTA = TMEM lanes
 constexpr int BK = 64;       // K elements per stage: one 128-byte swizzle span
-constexpr int BN = 224;      // output columns per tile
 constexpr int HC_MAX = 192;  // rank columns per down-projection chunk
 constexpr int RMAX = 576;
 constexpr uint32_t A_BYTES = BM * BK * 2;  // 16 KiB: this CTA's x tile
 constexpr uint32_t TMEM_COLS = 512;
 constexpr uint32_t ACC_COL = 0;
-constexpr uint32_t H_COL = BN;
 constexpr int NUM_THREADS = 320;  // producer, MMA, 8 epilogue warps
 constexpr int EPI_WARPS = 8;      // two per TMEM lane quarter, one per half tile
-constexpr int HALF_N = BN / 2;    // accumulator columns per epilogue warp
 constexpr int MAX_STAGES = 8;
 constexpr uint64_t TEARDOWN_LIMIT_NS = 200ull * 1000ull * 1000ull;
 constexpr size_t kMaxSmem = 232448;  // sm_100 opt-in maximum per block
 
-static_assert(H_COL + RMAX / 2 <= TMEM_COLS, "h does not fit next to the accumulator");
+constexpr uint32_t H_TILE_BYTES = BM * BK * 2;  // 16 KiB: 64 ranks of h for 128 rows
 
 // Per-variant constants.  PAIR = false: single-SM tcgen05.mma, 128-row
-// panels, each CTA loads whole B tiles.  PAIR = true: CTA pairs issue
-// tcgen05.mma.cta_group::2 over 256-row panels; each CTA holds 128 rows and
-// loads half of every B tile.
+// panels, 128 x 224 tiles, each CTA loads whole B tiles; TMEM holds the
+// accumulator (224 columns) and all 576 ranks of h (288 columns).
+// PAIR = true: CTA pairs issue tcgen05.mma.cta_group::2 over 256-row panels
+// with 256 x 256 tiles; each CTA holds 128 rows and loads half of every B
+// tile.  TMEM then holds the 256-column accumulator and ranks [0, 512) of h;
+// ranks [512, 576) live in a 16 KiB shared-memory tile (the up-projection
+// reads them from there as an ordinary shared-memory A operand), which costs
+// one stage of the ring but gives every stage 7 % more work per byte.
 template <bool PAIR>
 struct Cfg {
-  static constexpr uint32_t B_ROWS = PAIR ? BN / 2 : BN;  // W / B_cat rows a CTA loads
+  static constexpr int BN = PAIR ? 256 : 224;               // output columns per tile
+  static constexpr uint32_t H_COL = (uint32_t)BN;            // first TMEM column of h
+  static constexpr int R_TMEM = (int)(TMEM_COLS - BN) * 2;  // ranks of h held in TMEM
+  static constexpr bool H_SMEM = R_TMEM < RMAX;              // the rest in shared memory
+  static constexpr int HALF_N = BN / 2;                      // accumulator columns per epilogue warp
+  static constexpr uint32_t B_ROWS = PAIR ? BN / 2 : BN;    // W / B_cat rows a CTA loads
   static constexpr uint32_t B_BYTES = B_ROWS * BK * 2;
   static constexpr uint32_t STAGE = A_BYTES + B_BYTES;
   static constexpr int MMA_M = PAIR ? 2 * BM : BM;
   static constexpr int PANEL = PAIR ? 2 * BM : BM;
   static_assert(STAGE % 1024 == 0, "stages must stay 1024-byte aligned");
   static_assert((PAIR ? HC_MAX / 2 : HC_MAX) * BK * 2 <= B_BYTES, "A_cat chunk tile must fit the B slot");
+  static_assert(RMAX - R_TMEM <= BK, "ranks beyond TMEM must fit one shared-memory K block");
+  static_assert(R_TMEM % BK == 0, "the TMEM / shared-memory split of h must fall on a K block");
+  static_assert(HALF_N % 16 == 0 && HC_MAX <= BN, "epilogue and chunk widths");
 };
 
 struct Control {
@@ -116,6 +126,7 @@ struct Args {
   int stages;
   uint32_t staging_stride;  // bytes per staging row; the rows live at ring offset 0
   uint32_t control_off;     // byte offset of the Control block
+  uint32_t h_tile_off;      // byte offset of the shared-memory tile of h (pair variant)
   unsigned long long wait_limit_ns;
 };
 
@@ -253,7 +264,7 @@ __device__ void run_producer(const CUtensorMap* tm_x, const CUtensorMap* tm_w, c
       fence_proxy_async_smem();
     }
     for (int t = member; ok && t < a.n_tiles; t += a.group, ++sweep) {
-      const int n0 = t * BN + half * (int)C::B_ROWS;
+      const int n0 = t * C::BN + half * (int)C::B_ROWS;
       for (int i = 0; i < a.k_blocks; ++i) {
         const int kb = (sweep & 1) ? a.k_blocks - 1 - i : i;
         if (!wait_bounded(empty0 + 8 * stage, phase ^ 1, a.wait_limit_ns, abort_flag)) {
@@ -313,7 +324,7 @@ __device__ void run_mma(const Args& a, Control* ctl, uint32_t smem_base, uint32_
   const uint32_t acc_full = smem_u32(&ctl->acc_full);
   const uint32_t acc_empty = smem_u32(&ctl->acc_empty);
   const uint32_t idesc_h = idesc_bf16_f32(C::MMA_M, a.chunk_n);
-  constexpr uint32_t idesc_y = idesc_bf16_f32(C::MMA_M, BN);
+  constexpr uint32_t idesc_y = idesc_bf16_f32(C::MMA_M, C::BN);
   const uint32_t d_acc = tmem + ACC_COL;
   auto commit = [&](uint32_t bar) {
     if constexpr (PAIR) {
@@ -389,10 +400,17 @@ __device__ void run_mma(const Args& a, Control* ctl, uint32_t smem_base, uint32_
         tc_fence_after();
         const uint32_t sa = smem_base + stage * C::STAGE;
         const uint64_t db = sw128_kmajor_desc(sa + A_BYTES);
+        if (!C::H_SMEM || rb * BK < C::R_TMEM) {
 #pragma unroll
-        for (int kk = 0; kk < BK / 16; ++kk) {
-          // 16 ranks of h = 8 packed columns.
-          mma_ts(tmem + H_COL + (uint32_t)(rb * (BK / 2) + kk * 8), db + 2 * kk);
+          for (int kk = 0; kk < BK / 16; ++kk) {
+            // 16 ranks of h = 8 packed columns.
+            mma_ts(tmem + C::H_COL + (uint32_t)(rb * (BK / 2) + kk * 8), db + 2 * kk);
+          }
+        } else {
+          // The last 64 ranks of h: A from the shared-memory tile.
+          const uint64_t dh = sw128_kmajor_desc(smem_base + a.h_tile_off);
+#pragma unroll
+          for (int kk = 0; kk < BK / 16; ++kk) mma_ss(dh + 2 * kk, db + 2 * kk, idesc_y, 1u);
         }
         commit(empty0 + 8 * stage);
         advance(stage, phase, stages);
@@ -409,65 +427,111 @@ __device__ void run_mma(const Args& a, Control* ctl, uint32_t smem_base, uint32_
 
 // ---------------------------------------------------------------------------
 // Epilogue helpers (one warp: TMEM lanes of its quarter, half of the blocks).
+//
+// h storage: ranks [0, R_TMEM) as packed bf16 pairs in TMEM columns H_COL..;
+// ranks [R_TMEM, R) (pair variant only) in the shared-memory tile, one
+// 128-byte row per token row, K-major with the 128-byte swizzle (16-byte
+// chunk c of row r sits at chunk c ^ (r mod 8)), as the MMA reads it.
+// Ranks move in blocks of 16 (8 packed words) or 8 (4 words); a block never
+// straddles R_TMEM (the host only launches chunkings whose blocks start on a
+// multiple of 16 when part of h is in shared memory).
 // ---------------------------------------------------------------------------
-// FP32 accumulator columns [0, count) = ranks first .. first+count-1 ->
-// bf16 pairs in the h columns.  count is a multiple of 8.
-__device__ __forceinline__ void acc_to_h(uint32_t lane_base, int first, int count, int half) {
+struct HRow {
+  uint32_t lane_base;  // TMEM address of this warp's lane quarter
+  uint32_t tile_row;   // shared address of this thread's row of the h tile
+  uint32_t sw;         // row mod 8
+};
+
+template <bool PAIR, int WORDS>
+__device__ __forceinline__ void h_put(const HRow& h, int r0, const uint32_t (&v)[WORDS]) {
+  using C = Cfg<PAIR>;
+  if (!C::H_SMEM || r0 < C::R_TMEM) {
+    if constexpr (WORDS == 8) {
+      tmem_st_32x32b_x8(h.lane_base + C::H_COL + (uint32_t)(r0 / 2), v);
+    } else {
+      tmem_st_32x32b_x4(h.lane_base + C::H_COL + (uint32_t)(r0 / 2), v);
+    }
+  } else {
+    const uint32_t c = (uint32_t)(r0 - C::R_TMEM) / 8;
+    st_shared_v4(h.tile_row + ((c ^ h.sw) << 4), v[0], v[1], v[2], v[3]);
+    if constexpr (WORDS == 8) st_shared_v4(h.tile_row + (((c + 1) ^ h.sw) << 4), v[4], v[5], v[6], v[7]);
+  }
+}
+
+template <bool PAIR, int WORDS>
+__device__ __forceinline__ void h_get(const HRow& h, int r0, uint32_t (&v)[WORDS]) {
+  using C = Cfg<PAIR>;
+  if (!C::H_SMEM || r0 < C::R_TMEM) {
+    if constexpr (WORDS == 8) {
+      tmem_ld_32x32b_x8(h.lane_base + C::H_COL + (uint32_t)(r0 / 2), v);
+    } else {
+      tmem_ld_32x32b_x4(h.lane_base + C::H_COL + (uint32_t)(r0 / 2), v);
+    }
+    tmem_wait_ld();
+  } else {
+    const uint32_t c = (uint32_t)(r0 - C::R_TMEM) / 8;
+    ld_shared_v4(h.tile_row + ((c ^ h.sw) << 4), v[0], v[1], v[2], v[3]);
+    if constexpr (WORDS == 8) ld_shared_v4(h.tile_row + (((c + 1) ^ h.sw) << 4), v[4], v[5], v[6], v[7]);
+  }
+}
+
+// FP32 accumulator columns [0, count) = ranks first .. first+count-1 -> bf16
+// pairs in h.  count is a multiple of 8.
+template <bool PAIR>
+__device__ __forceinline__ void acc_to_h(const HRow& h, int first, int count, int half) {
   const int full_blocks = count / 16;
   for (int b = half; b < full_blocks; b += 2) {
     uint32_t v[16];
-    tmem_ld_32x32b_x16(lane_base + ACC_COL + 16 * b, v);
+    tmem_ld_32x32b_x16(h.lane_base + ACC_COL + 16 * b, v);
     tmem_wait_ld();
     uint32_t packed[8];
 #pragma unroll
     for (int i = 0; i < 8; ++i) packed[i] = pack_bf16x2(__uint_as_float(v[2 * i]), __uint_as_float(v[2 * i + 1]));
-    tmem_st_32x32b_x8(lane_base + H_COL + (uint32_t)((first + 16 * b) / 2), packed);
+    h_put<PAIR, 8>(h, first + 16 * b, packed);
   }
   if ((count % 16) && ((full_blocks & 1) == half)) {
     uint32_t v[8];
-    tmem_ld_32x32b_x8(lane_base + ACC_COL + 16 * full_blocks, v);
+    tmem_ld_32x32b_x8(h.lane_base + ACC_COL + 16 * full_blocks, v);
     tmem_wait_ld();
     uint32_t packed[4];
 #pragma unroll
     for (int i = 0; i < 4; ++i) packed[i] = pack_bf16x2(__uint_as_float(v[2 * i]), __uint_as_float(v[2 * i + 1]));
-    tmem_st_32x32b_x4(lane_base + H_COL + (uint32_t)((first + 16 * full_blocks) / 2), packed);
+    h_put<PAIR, 4>(h, first + 16 * full_blocks, packed);
   }
   tmem_wait_st();
 }
 
-// This member's slice of h (pairs s0/2 .. ) from TMEM into its staging row.
-__device__ __forceinline__ void h_to_staging(uint32_t lane_base, int s0, int slice, int half, uint32_t row) {
-  const int cols = slice / 2;  // multiple of 4
-  const uint32_t src = lane_base + H_COL + (uint32_t)(s0 / 2);
-  for (int b = half; b < cols / 8; b += 2) {
+// This member's slice of h (ranks s0 .. s0 + slice - 1) into its staging row.
+template <bool PAIR>
+__device__ __forceinline__ void h_to_staging(const HRow& h, int s0, int slice, int half, uint32_t row) {
+  const int blocks = slice / 16;
+  for (int b = half; b < blocks; b += 2) {
     uint32_t v[8];
-    tmem_ld_32x32b_x8(src + 8 * b, v);
-    tmem_wait_ld();
+    h_get<PAIR, 8>(h, s0 + 16 * b, v);
     st_shared_v4(row + 32u * b, v[0], v[1], v[2], v[3]);
     st_shared_v4(row + 32u * b + 16, v[4], v[5], v[6], v[7]);
   }
-  if ((cols % 8) && (((cols / 8) & 1) == half)) {
+  if ((slice % 16) && ((blocks & 1) == half)) {
     uint32_t v[4];
-    tmem_ld_32x32b_x4(src + 8 * (cols / 8), v);
-    tmem_wait_ld();
-    st_shared_v4(row + 32u * (cols / 8), v[0], v[1], v[2], v[3]);
+    h_get<PAIR, 4>(h, s0 + 16 * blocks, v);
+    st_shared_v4(row + 32u * blocks, v[0], v[1], v[2], v[3]);
   }
 }
 
-// A peer's staged slice (cluster address of its row) into this CTA's h columns.
-__device__ __forceinline__ void staging_to_h(uint32_t lane_base, int s0, int slice, int half, uint32_t remote_row) {
-  const int cols = slice / 2;
-  const uint32_t dst = lane_base + H_COL + (uint32_t)(s0 / 2);
-  for (int b = half; b < cols / 8; b += 2) {
+// A peer's staged slice (cluster address of its row) into this CTA's h.
+template <bool PAIR>
+__device__ __forceinline__ void staging_to_h(const HRow& h, int s0, int slice, int half, uint32_t remote_row) {
+  const int blocks = slice / 16;
+  for (int b = half; b < blocks; b += 2) {
     uint32_t v[8];
     ld_shared_cluster_v4(remote_row + 32u * b, v[0], v[1], v[2], v[3]);
     ld_shared_cluster_v4(remote_row + 32u * b + 16, v[4], v[5], v[6], v[7]);
-    tmem_st_32x32b_x8(dst + 8 * b, v);
+    h_put<PAIR, 8>(h, s0 + 16 * b, v);
   }
-  if ((cols % 8) && (((cols / 8) & 1) == half)) {
+  if ((slice % 16) && ((blocks & 1) == half)) {
     uint32_t v[4];
-    ld_shared_cluster_v4(remote_row + 32u * (cols / 8), v[0], v[1], v[2], v[3]);
-    tmem_st_32x32b_x4(dst + 8 * (cols / 8), v);
+    ld_shared_cluster_v4(remote_row + 32u * blocks, v[0], v[1], v[2], v[3]);
+    h_put<PAIR, 4>(h, s0 + 16 * blocks, v);
   }
 }
 
@@ -491,22 +555,34 @@ __device__ void run_epilogue(const Args& a, Control* ctl, uint32_t smem_base, ui
   const uint32_t slice_free = smem_u32(&ctl->slice_free);
   const uint32_t epi_sync = smem_u32(&ctl->epi_sync);
   const uint32_t my_row = smem_base + (uint32_t)row_in_tile * a.staging_stride;
+  HRow hr;
+  hr.lane_base = lane_base;
+  hr.tile_row = smem_base + a.h_tile_off + (uint32_t)row_in_tile * (BK * 2);
+  hr.sw = (uint32_t)row_in_tile & 7u;
   auto peer_rank = [&](int c) { return (uint32_t)(PAIR ? 2 * c + parity : c); };
   uint32_t acc_phase = 0;
   uint32_t it = 0;
   bool ok = true;
   // y is written once and not read here: let it leave L2 first.
   const uint64_t pol_y = l2_policy_evict_first();
-  // Hands the accumulator back to the MMA issuer.  Every lane's tcgen05.ld has
-  // completed (tcgen05.wait::ld) before lane 0 arrives, and the arrival
-  // publishes no data, so the pair form arrives relaxed: a release at cluster
-  // scope measured ~1 us per tile, all of it on the MMA's critical path.
-  auto release_acc = [&]() {
+  // Hands the accumulator back to the MMA issuer.  After a tile (publish =
+  // false) every lane's tcgen05.ld has completed (tcgen05.wait::ld) before
+  // lane 0 arrives and the arrival publishes no data, so the pair form arrives
+  // relaxed: a release at cluster scope measured ~1 us per tile, all of it on
+  // the MMA's critical path.  After a chunk of h (publish = true) the arrival
+  // publishes h -- TMEM columns and, for pairs, shared-memory rows that the
+  // leader's MMAs read through the async proxy -- so it is a release.
+  auto release_acc = [&](bool publish) {
+    if (publish && C::H_SMEM) fence_proxy_async_smem();
     tc_fence_before();
     __syncwarp();
     if (lane == 0) {
       if constexpr (PAIR) {
-        mbar_arrive_remote_relaxed(acc_empty);
+        if (publish) {
+          mbar_arrive_remote(acc_empty);
+        } else {
+          mbar_arrive_remote_relaxed(acc_empty);
+        }
       } else {
         mbar_arrive(acc_empty);
       }
@@ -521,7 +597,7 @@ __device__ void run_epilogue(const Args& a, Control* ctl, uint32_t smem_base, ui
       tc_fence_after();
       int first, count;
       chunk_ranks(a, member, j, first, count);
-      acc_to_h(lane_base, first, count, half);
+      acc_to_h<PAIR>(hr, first, count, half);
       if (a.group > 1 && j == a.n_chunks - 1) {
         // Swap slices with the other members of the group: stage this slice
         // at the start of the (idle) ring, wait for every member's, copy the
@@ -535,7 +611,7 @@ __device__ void run_epilogue(const Args& a, Control* ctl, uint32_t smem_base, ui
         if (!ok) break;
         tc_fence_after();
         fence_proxy_async_smem();
-        h_to_staging(lane_base, member * a.slice, a.slice, half, my_row);
+        h_to_staging<PAIR>(hr, member * a.slice, a.slice, half, my_row);
         __syncwarp();
         if (lane == 0) {
           for (int c = 0; c < a.group; ++c) mbar_arrive_remote(mapa_shared(slice_ready, peer_rank(c)));
@@ -543,7 +619,7 @@ __device__ void run_epilogue(const Args& a, Control* ctl, uint32_t smem_base, ui
         ok = __all_sync(0xffffffffu, wait_bounded(slice_ready, it & 1, a.wait_limit_ns, abort_flag, true));
         if (!ok) break;
         for (int c = 0; c < a.group; ++c) {
-          if (c != member) staging_to_h(lane_base, c * a.slice, a.slice, half, mapa_shared(my_row, peer_rank(c)));
+          if (c != member) staging_to_h<PAIR>(hr, c * a.slice, a.slice, half, mapa_shared(my_row, peer_rank(c)));
         }
         tmem_wait_st();
         __syncwarp();
@@ -551,45 +627,40 @@ __device__ void run_epilogue(const Args& a, Control* ctl, uint32_t smem_base, ui
           for (int c = 0; c < a.group; ++c) mbar_arrive_remote(mapa_shared(slice_free, peer_rank(c)));
         }
       }
-      release_acc();
+      release_acc(true);
     }
     for (int t = member; ok && t < a.n_tiles; t += a.group) {
       ok = __all_sync(0xffffffffu, wait_bounded(acc_full, acc_phase, a.wait_limit_ns, abort_flag));
       if (!ok) break;
       tc_fence_after();
-      // Pull this warp's 112 accumulator columns into registers and hand the
-      // accumulator back at once, so the next tile's MMAs overlap the
+      // Pull this warp's HALF_N accumulator columns into registers and hand
+      // the accumulator back at once, so the next tile's MMAs overlap the
       // conversion and the stores below.
-      const uint32_t src = lane_base + ACC_COL + (uint32_t)(half * HALF_N);
-      uint32_t v0[32], v1[32], v2[32], v3[16];
-      tmem_ld_32x32b_x32(src, v0);
-      tmem_ld_32x32b_x32(src + 32, v1);
-      tmem_ld_32x32b_x32(src + 64, v2);
-      tmem_ld_32x32b_x16(src + 96, v3);
+      constexpr int N32 = C::HALF_N / 32;
+      constexpr bool TAIL16 = (C::HALF_N % 32) != 0;
+      const uint32_t src = lane_base + ACC_COL + (uint32_t)(half * C::HALF_N);
+      uint32_t v[N32 + (TAIL16 ? 1 : 0)][32];
+#pragma unroll
+      for (int i = 0; i < N32; ++i) tmem_ld_32x32b_x32(src + 32 * i, v[i]);
+      if constexpr (TAIL16) tmem_ld_32x32b_x16(src + 32 * N32, *reinterpret_cast<uint32_t(*)[16]>(v[N32]));
       tmem_wait_ld();
-      release_acc();
+      release_acc(false);
 
       const int64_t row = m0 + row_in_tile;
-      const int col0 = t * BN + half * HALF_N;
+      const int col0 = t * C::BN + half * C::HALF_N;
       if (row < a.M) {
         uint16_t* dst_row = a.y + row * (int64_t)a.N;
-        auto store8 = [&](int g, const uint32_t* v) {
+#pragma unroll
+        for (int g = 0; g < C::HALF_N / 8; ++g) {
           const int col = col0 + 8 * g;
+          const uint32_t* w = &v[g / 4][8 * (g % 4)];
           if (col < a.N) {
-            st_global_v4_hint(dst_row + col, pack_bf16x2(__uint_as_float(v[0]), __uint_as_float(v[1])),
-                              pack_bf16x2(__uint_as_float(v[2]), __uint_as_float(v[3])),
-                              pack_bf16x2(__uint_as_float(v[4]), __uint_as_float(v[5])),
-                              pack_bf16x2(__uint_as_float(v[6]), __uint_as_float(v[7])), pol_y);
+            st_global_v4_hint(dst_row + col, pack_bf16x2(__uint_as_float(w[0]), __uint_as_float(w[1])),
+                              pack_bf16x2(__uint_as_float(w[2]), __uint_as_float(w[3])),
+                              pack_bf16x2(__uint_as_float(w[4]), __uint_as_float(w[5])),
+                              pack_bf16x2(__uint_as_float(w[6]), __uint_as_float(w[7])), pol_y);
           }
-        };
-#pragma unroll
-        for (int g = 0; g < 4; ++g) store8(g, v0 + 8 * g);
-#pragma unroll
-        for (int g = 0; g < 4; ++g) store8(4 + g, v1 + 8 * g);
-#pragma unroll
-        for (int g = 0; g < 4; ++g) store8(8 + g, v2 + 8 * g);
-#pragma unroll
-        for (int g = 0; g < 2; ++g) store8(12 + g, v3 + 8 * g);
+        }
       }
     }
   }
@@ -715,7 +786,7 @@ bool make_map(PFN_cuTensorMapEncodeTiled_v12000 enc, CUtensorMap* m, const void*
 // shared memory goes to the ring.
 struct Geometry {
   int group = 1, slice = 0, n_chunks = 0, chunk_valid = 0, chunk_n = 16, stages = 0;
-  uint32_t staging_stride = 0, control_off = 0;
+  uint32_t staging_stride = 0, control_off = 0, h_tile_off = 0;
   size_t smem = 0;
 };
 
@@ -732,13 +803,18 @@ bool make_geometry(int group, int R, Geometry* g) {
     g->chunk_n = (g->chunk_valid + 15) / 16 * 16;
     if (g->chunk_n > HC_MAX) return false;
     g->staging_stride = (uint32_t)(2 * g->slice + 16);
+    // Part of h in shared memory: every block of 16 ranks must fall wholly on
+    // one side of the split (slices and chunks start on multiples of 16).
+    if (C::H_SMEM && R > C::R_TMEM && (g->slice % 16 || g->chunk_valid % 16)) return false;
   }
-  const size_t fixed = 1024 + sizeof(Control);
+  const uint32_t h_tile = C::H_SMEM ? H_TILE_BYTES : 0u;
+  const size_t fixed = 1024 + h_tile + sizeof(Control);
   g->stages = (int)((kMaxSmem - fixed) / C::STAGE);
   if (g->stages > MAX_STAGES) g->stages = MAX_STAGES;
   if (g->stages < 2) return false;
   if (group > 1 && (size_t)BM * g->staging_stride > (size_t)g->stages * C::STAGE) return false;
-  g->control_off = (uint32_t)g->stages * C::STAGE;
+  g->h_tile_off = (uint32_t)g->stages * C::STAGE;  // 1024-aligned: stages are
+  g->control_off = g->h_tile_off + h_tile;
   g->smem = 1024 + (size_t)g->control_off + sizeof(Control);
   return true;
 }
@@ -823,7 +899,7 @@ cudaError_t launch_variant(const LinearLaunch& p, cudaStream_t s, int dev, int c
   args.N = p.N;
   args.R = p.R;
   args.num_panels = (int)((p.M + C::PANEL - 1) / C::PANEL);
-  args.n_tiles = (p.N + BN - 1) / BN;
+  args.n_tiles = (p.N + C::BN - 1) / C::BN;
   args.k_blocks = p.K / BK;
   args.r_blocks = p.R / BK;
   args.group = group;
@@ -834,6 +910,7 @@ cudaError_t launch_variant(const LinearLaunch& p, cudaStream_t s, int dev, int c
   args.stages = geo.stages;
   args.staging_stride = geo.staging_stride;
   args.control_off = geo.control_off;
+  args.h_tile_off = geo.h_tile_off;
   args.wait_limit_ns = p.wait_limit_ns;
   const void* kernel = (const void*)k_lora_linear<PAIR>;
   int clusters = max_active_clusters(kernel, PAIR ? 2 : 1, dev, cluster, geo.smem, p.sm_count);
@@ -878,20 +955,18 @@ cudaError_t launch_lora_linear(const LinearLaunch& p, cudaStream_t s, bool* driv
   if (e != cudaSuccess) return e;
   // Variant and cluster size (both process-wide overrides for tuning).  The
   // automatic choice follows sustained (power-capped) sweeps on B200: private
-  // panels for small K; SM pairs, one or two per panel, for K up to 8192;
-  // single-SM pairs of CTAs beyond, where the panels' x no longer fits L2
-  // either way and the SM pairs' extra DRAM traffic costs clock.
+  // single-SM panels for small K; above, SM pairs with 256 x 256 tiles, one
+  // pair per panel up to K = 4096 and two beyond (clusters of 4: the panel's
+  // x is fetched once for four SMs).
   int variant = g_variant_override;
   int cluster = g_cluster_override;
   if (variant == 0) {
     if (p.K <= 2048 || cluster == 1) {
       variant = 1;
       if (cluster == 0) cluster = 1;
-    } else if (p.K <= 8192) {
+    } else {
       variant = 2;
       if (cluster == 0) cluster = p.K <= 4096 ? 2 : 4;
-    } else {
-      variant = 1;
     }
   }
   if (variant == 1) {
