@@ -67,6 +67,11 @@ constexpr uint64_t TEARDOWN_LIMIT_NS = 200ull * 1000ull * 1000ull;
 constexpr size_t kMaxSmem = 232448;  // sm_100 opt-in maximum per block
 
 constexpr uint32_t H_TILE_BYTES = BM * BK * 2;  // 16 KiB: 64 ranks of h for 128 rows
+// Pair variant: y leaves through a TMA store, staged per epilogue warp in
+// 32 x 32 bf16 boxes (64-byte rows, 64-byte swizzle).
+constexpr int Y_BOX = 32;
+constexpr uint32_t Y_WARP_BYTES = Y_BOX * Y_BOX * 2;              // 2 KiB
+constexpr uint32_t Y_STAGE_BYTES = 8 * Y_WARP_BYTES;              // 16 KiB for the 8 epilogue warps
 
 // Per-variant constants.  PAIR = false: single-SM tcgen05.mma, 128-row
 // panels, 128 x 224 tiles, each CTA loads whole B tiles; TMEM holds the
@@ -127,6 +132,7 @@ struct Args {
   uint32_t staging_stride;  // bytes per staging row; the rows live at ring offset 0
   uint32_t control_off;     // byte offset of the Control block
   uint32_t h_tile_off;      // byte offset of the shared-memory tile of h (pair variant)
+  uint32_t y_stage_off;     // byte offset of the y staging boxes (pair variant)
   unsigned long long wait_limit_ns;
 };
 
@@ -540,7 +546,7 @@ __device__ __forceinline__ void staging_to_h(const HRow& h, int s0, int slice, i
 // handles half (w - 2) / 4 of the columns.
 // ---------------------------------------------------------------------------
 template <bool PAIR>
-__device__ void run_epilogue(const Args& a, Control* ctl, uint32_t smem_base, uint32_t tmem, uint32_t crank,
+__device__ void run_epilogue(const CUtensorMap* tm_y, const Args& a, Control* ctl, uint32_t smem_base, uint32_t tmem, uint32_t crank,
                              uint32_t cid, uint32_t ncl, int warp, int lane, volatile int* abort_flag) {
   using C = Cfg<PAIR>;
   const int q = warp & 3;
@@ -646,31 +652,63 @@ __device__ void run_epilogue(const Args& a, Control* ctl, uint32_t smem_base, ui
       tmem_wait_ld();
       release_acc(false);
 
-      const int64_t row = m0 + row_in_tile;
       const int col0 = t * C::BN + half * C::HALF_N;
-      if (row < a.M) {
-        uint16_t* dst_row = a.y + row * (int64_t)a.N;
+      if constexpr (PAIR) {
+        // 32 x 32 boxes through this warp's staging buffer: convert, write
+        // this lane's 64-byte row (16-byte chunk c at c ^ ((row / 2) mod 4),
+        // the 64-byte swizzle), hand the box to a TMA store, and rewrite the
+        // buffer only once that store has read it.
+        const uint32_t buf = smem_base + a.y_stage_off + (uint32_t)(warp - 2) * Y_WARP_BYTES;
+        const uint32_t my = buf + (uint32_t)lane * (Y_BOX * 2);
+        const uint32_t sw = ((uint32_t)lane >> 1) & 3u;
 #pragma unroll
-        for (int g = 0; g < C::HALF_N / 8; ++g) {
-          const int col = col0 + 8 * g;
-          const uint32_t* w = &v[g / 4][8 * (g % 4)];
-          if (col < a.N) {
-            st_global_v4_hint(dst_row + col, pack_bf16x2(__uint_as_float(w[0]), __uint_as_float(w[1])),
-                              pack_bf16x2(__uint_as_float(w[2]), __uint_as_float(w[3])),
-                              pack_bf16x2(__uint_as_float(w[4]), __uint_as_float(w[5])),
-                              pack_bf16x2(__uint_as_float(w[6]), __uint_as_float(w[7])), pol_y);
+        for (int c4 = 0; c4 < C::HALF_N / Y_BOX; ++c4) {
+          if (lane == 0) bulk_wait_group_read0();
+          __syncwarp();
+#pragma unroll
+          for (int c = 0; c < 4; ++c) {
+            const uint32_t* w = &v[c4][8 * c];
+            st_shared_v4(my + (((uint32_t)c ^ sw) << 4), pack_bf16x2(__uint_as_float(w[0]), __uint_as_float(w[1])),
+                         pack_bf16x2(__uint_as_float(w[2]), __uint_as_float(w[3])),
+                         pack_bf16x2(__uint_as_float(w[4]), __uint_as_float(w[5])),
+                         pack_bf16x2(__uint_as_float(w[6]), __uint_as_float(w[7])));
+          }
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) {
+            tma_store_2d_hint(tm_y, buf, col0 + Y_BOX * c4, (int)(m0 + 32 * q), pol_y);
+            bulk_commit_group();
+          }
+        }
+      } else {
+        const int64_t row = m0 + row_in_tile;
+        if (row < a.M) {
+          uint16_t* dst_row = a.y + row * (int64_t)a.N;
+#pragma unroll
+          for (int g = 0; g < C::HALF_N / 8; ++g) {
+            const int col = col0 + 8 * g;
+            const uint32_t* w = &v[g / 4][8 * (g % 4)];
+            if (col < a.N) {
+              st_global_v4_hint(dst_row + col, pack_bf16x2(__uint_as_float(w[0]), __uint_as_float(w[1])),
+                                pack_bf16x2(__uint_as_float(w[2]), __uint_as_float(w[3])),
+                                pack_bf16x2(__uint_as_float(w[4]), __uint_as_float(w[5])),
+                                pack_bf16x2(__uint_as_float(w[6]), __uint_as_float(w[7])), pol_y);
+            }
           }
         }
       }
     }
   }
+  // The y stores of this warp have completed before the CTA can exit.
+  if (PAIR && lane == 0) bulk_wait_group0();
+  __syncwarp();
 }
 
 template <bool PAIR>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     k_lora_linear(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_w,
                   const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b,
-                  const Args args) {
+                  const __grid_constant__ CUtensorMap tm_y, const Args args) {
   extern __shared__ uint8_t smem_raw[];
   // Dynamic shared memory starts at the same offset in every CTA, so after
   // rounding up to 1 KiB the layout (and every mapa'd address) matches.
@@ -699,6 +737,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     fence_mbarrier_init();
     tma_prefetch_desc(&tm_x);
     tma_prefetch_desc(&tm_w);
+    if (PAIR) tma_prefetch_desc(&tm_y);
     if (args.R > 0) {
       tma_prefetch_desc(&tm_a);
       tma_prefetch_desc(&tm_b);
@@ -727,7 +766,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     if (lane == 0 && issues_mma) run_mma<PAIR>(args, ctl, smem_base, tmem, crank, cid, ncl, abort_flag);
     __syncwarp();
   } else {
-    run_epilogue<PAIR>(args, ctl, smem_base, tmem, crank, cid, ncl, warp, lane, abort_flag);
+    run_epilogue<PAIR>(&tm_y, args, ctl, smem_base, tmem, crank, cid, ncl, warp, lane, abort_flag);
   }
 
   tc_fence_before();
@@ -781,12 +820,25 @@ bool make_map(PFN_cuTensorMapEncodeTiled_v12000 enc, CUtensorMap* m, const void*
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// Row-major bf16 y [rows, cols] written in 32 x 32 boxes from 64-byte-swizzled
+// shared memory; the store clips rows and columns outside the matrix.
+bool make_store_map(PFN_cuTensorMapEncodeTiled_v12000 enc, CUtensorMap* m, void* base, uint64_t cols,
+                    uint64_t rows) {
+  cuuint64_t dims[2] = {cols, rows};
+  cuuint64_t strides[1] = {cols * 2};
+  cuuint32_t box[2] = {(cuuint32_t)Y_BOX, (cuuint32_t)Y_BOX};
+  cuuint32_t elem_strides[2] = {1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, base, dims, strides, box, elem_strides,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 // Launch geometry: down-projection chunking and stage count.  The h
 // exchange of a group reuses the start of the stage ring, so every stage of
 // shared memory goes to the ring.
 struct Geometry {
   int group = 1, slice = 0, n_chunks = 0, chunk_valid = 0, chunk_n = 16, stages = 0;
-  uint32_t staging_stride = 0, control_off = 0, h_tile_off = 0;
+  uint32_t staging_stride = 0, control_off = 0, h_tile_off = 0, y_stage_off = 0;
   size_t smem = 0;
 };
 
@@ -808,13 +860,15 @@ bool make_geometry(int group, int R, Geometry* g) {
     if (C::H_SMEM && R > C::R_TMEM && (g->slice % 16 || g->chunk_valid % 16)) return false;
   }
   const uint32_t h_tile = C::H_SMEM ? H_TILE_BYTES : 0u;
-  const size_t fixed = 1024 + h_tile + sizeof(Control);
+  const uint32_t y_stage = PAIR ? Y_STAGE_BYTES : 0u;
+  const size_t fixed = 1024 + h_tile + y_stage + sizeof(Control);
   g->stages = (int)((kMaxSmem - fixed) / C::STAGE);
   if (g->stages > MAX_STAGES) g->stages = MAX_STAGES;
   if (g->stages < 2) return false;
   if (group > 1 && (size_t)BM * g->staging_stride > (size_t)g->stages * C::STAGE) return false;
   g->h_tile_off = (uint32_t)g->stages * C::STAGE;  // 1024-aligned: stages are
-  g->control_off = g->h_tile_off + h_tile;
+  g->y_stage_off = g->h_tile_off + h_tile;
+  g->control_off = g->y_stage_off + y_stage;
   g->smem = 1024 + (size_t)g->control_off + sizeof(Control);
   return true;
 }
@@ -879,9 +933,16 @@ cudaError_t launch_variant(const LinearLaunch& p, cudaStream_t s, int dev, int c
   Geometry geo;
   if (!make_geometry<PAIR>(group, p.R, &geo)) return cudaErrorInvalidConfiguration;
   const uint32_t a_rows = PAIR ? (uint32_t)geo.chunk_n / 2 : (uint32_t)geo.chunk_n;
-  CUtensorMap tm_x, tm_w, tm_a, tm_b;
+  CUtensorMap tm_x, tm_w, tm_a, tm_b, tm_y;
   bool ok = make_map(enc, &tm_x, p.x, (uint64_t)p.K, (uint64_t)p.M, BM) &&
             make_map(enc, &tm_w, p.W, (uint64_t)p.K, (uint64_t)p.N, C::B_ROWS);
+  if (ok) {
+    if (PAIR) {
+      ok = make_store_map(enc, &tm_y, p.y, (uint64_t)p.N, (uint64_t)p.M);
+    } else {
+      tm_y = tm_x;  // never used: the single-SM epilogue stores directly
+    }
+  }
   if (ok && p.R > 0) {
     ok = make_map(enc, &tm_a, p.A_bf16, (uint64_t)p.K, (uint64_t)p.R, a_rows) &&
          make_map(enc, &tm_b, p.B_bf16, (uint64_t)p.R, (uint64_t)p.N, C::B_ROWS);
@@ -911,6 +972,7 @@ cudaError_t launch_variant(const LinearLaunch& p, cudaStream_t s, int dev, int c
   args.staging_stride = geo.staging_stride;
   args.control_off = geo.control_off;
   args.h_tile_off = geo.h_tile_off;
+  args.y_stage_off = geo.y_stage_off;
   args.wait_limit_ns = p.wait_limit_ns;
   const void* kernel = (const void*)k_lora_linear<PAIR>;
   int clusters = max_active_clusters(kernel, PAIR ? 2 : 1, dev, cluster, geo.smem, p.sm_count);
@@ -930,7 +992,7 @@ cudaError_t launch_variant(const LinearLaunch& p, cudaStream_t s, int dev, int c
   attr[0].val.clusterDim.z = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  void* params[5] = {&tm_x, &tm_w, &tm_a, &tm_b, &args};
+  void* params[6] = {&tm_x, &tm_w, &tm_a, &tm_b, &tm_y, &args};
   cudaError_t e = cudaLaunchKernelExC(&cfg, kernel, params);
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
