@@ -92,9 +92,10 @@ void lg_set_wait_limit_ns(uint64_t limit_ns);
  * LG_ERR_INVALID_ARG for other values. */
 lg_status lg_set_cluster_size(int g);
 
-/* MMA variant of lg_lora_linear: 1 = single-SM tcgen05.mma (128-row tiles),
- * 2 = SM-pair tcgen05.mma.cta_group::2 (256-row tiles, each SM loads half of
- * every B tile), 0 (the default) = chosen per shape.  Process-wide; for
+/* MMA variant of lg_lora_linear: 1 = single-SM tcgen05.mma (128 x 224
+ * tiles), 2 = SM-pair tcgen05.mma.cta_group::2 (256 x 256 tiles, each SM
+ * loads half of every B tile), 0 (the default) = chosen per shape (single-SM
+ * for K <= 2048, pairs beyond).  Process-wide; for
  * tuning and tests.  Returns LG_ERR_INVALID_ARG for other values. */
 lg_status lg_set_kernel_variant(int v);
 

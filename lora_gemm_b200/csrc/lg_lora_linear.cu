@@ -9,32 +9,36 @@
 // "三个步如何完成工作", rank 384 + 128 + 64 = 576 on 312 linear layers); the
 // pages give no kernel design, so everything below is this library's.
 //
-// Design (persistent; one CTA per SM; clusters of G CTAs share a panel):
-//   * A panel is 128 token rows (one TMEM lane per row).  The G CTAs of a
+// Design (persistent; one CTA per SM; clusters share a panel):
+//   * A panel is the token rows one CTA (single-SM variant: 128 rows, one
+//     TMEM lane per row) or one CTA pair (pair variant, tcgen05.mma
+//     cta_group::2: 256 rows, 128 per CTA) owns.  The G members of a
 //     thread-block cluster work on the same panel at the same time, so the
 //     panel of x is fetched from DRAM once and re-read from L2 by all of them
-//     while they split its N tiles (tile t goes to CTA t mod G).  With G = 1
-//     every SM owns a private panel, which suits small K; for large K the
-//     148 private panels would not fit in L2.
-//   * TMEM (512 columns x 128 lanes) holds the FP32 accumulator of one
-//     128 x 224 output tile in columns [0, 224) and the panel's rank-R
-//     intermediate h = x A_cat^T as packed bf16 pairs in columns
-//     [224, 224 + R/2) -- 288 columns for R = 576.  h never leaves the chip.
-//   * Phase A (per panel): each CTA of the cluster computes its slice of
-//     ceil(R/G) ranks of h (tcgen05.mma, A = x tile, B = A_cat tile, both in
-//     shared memory).  With G = 1 the epilogue writes h straight into TMEM;
-//     with G > 1 each CTA rounds its slice to bf16 into a shared-memory
-//     staging buffer, the CTAs signal each other through cluster-scope
+//     while they split its N tiles (tile t goes to member t mod G).
+//   * TMEM (512 columns x 128 lanes) holds the FP32 accumulator of one output
+//     tile and the panel's rank-R intermediate h = x A_cat^T as packed bf16
+//     pairs: single-SM 128 x 224 tiles, accumulator in columns [0, 224) and
+//     all 576 ranks of h in [224, 512); pairs 256 x 256 tiles, accumulator in
+//     [0, 256), ranks [0, 512) of h in [256, 512) and ranks [512, 576) in a
+//     16 KiB shared-memory tile.  h never leaves the chip.
+//   * Phase A (per panel): each member computes its slice of R/G ranks of h
+//     (tcgen05.mma, A = x tile, B = A_cat tile, both in shared memory).  With
+//     G = 1 the epilogue writes h straight into TMEM (and the shared tile);
+//     with G > 1 each member rounds its slice to bf16 into a shared-memory
+//     staging buffer, the members signal each other through cluster-scope
 //     mbarriers, and every CTA copies all G slices (its own and its peers',
-//     through distributed shared memory) into its own TMEM.
+//     through distributed shared memory) into its own h.
 //   * Phase B (per N tile): a K loop x W^T into the accumulator, then R/16
-//     more MMAs with A = h read straight from TMEM and B = the B_cat tile;
-//     the epilogue converts the tile to bf16 and stores it.
-//   * Warp roles: warp 0 issues TMA loads into a ring of 44 KiB stages
-//     (128-byte swizzled K-major tiles), warp 1 issues the MMAs (one thread)
-//     and owns the TMEM allocation, warps 2-9 are the epilogue: each pulls
-//     half of the tile's accumulator into registers, releases the TMEM
-//     accumulator to the next tile's MMAs, then converts and stores y.
+//     more MMAs with A = h read straight from TMEM (the last 64 ranks of the
+//     pair variant from the shared tile) and B = the B_cat tile; the epilogue
+//     converts the tile to bf16 and stores it (pairs: TMA stores).
+//   * Warp roles: warp 0 issues TMA loads into a ring of stages of 64 K
+//     elements (128-byte swizzled K-major tiles: 44 KiB single-SM, 32 KiB per
+//     CTA of a pair), warp 1 issues the MMAs (one thread) and owns the TMEM
+//     allocation, warps 2-9 are the epilogue: each pulls half of the tile's
+//     accumulator into registers, releases the TMEM accumulator to the next
+//     tile's MMAs, then converts and stores y.
 //   * Every mbarrier wait is bounded; on expiry the kernel records
 //     LG_ERR_DEVICE_TIMEOUT in the device error word, drains its own TMA
 //     copies and MMAs, frees its TMEM and returns.
