@@ -42,6 +42,7 @@
 //   * Every mbarrier wait is bounded; on expiry the kernel records
 //     LG_ERR_DEVICE_TIMEOUT in the device error word, drains its own TMA
 //     copies and MMAs, frees its TMEM and returns.
+#include <atomic>
 #include <cstdlib>
 #include <mutex>
 
@@ -877,8 +878,9 @@ bool make_geometry(int group, int R, Geometry* g) {
   return true;
 }
 
-int g_cluster_override = 0;  // 0: automatic (lg_set_cluster_size)
-int g_variant_override = 0;  // 0: automatic, 1: single-SM MMA, 2: SM-pair MMA
+// Process-wide tuning overrides; set from any host thread, read at launch.
+std::atomic<int> g_cluster_override{0};  // 0: automatic (lg_set_cluster_size)
+std::atomic<int> g_variant_override{0};  // 0: automatic, 1: single-SM MMA, 2: SM-pair MMA
 
 // Resident clusters of `cluster` CTAs of `kernel` on device `dev` (cached).
 int max_active_clusters(const void* kernel, int variant, int dev, int cluster, size_t smem, int sm_count) {
@@ -1004,8 +1006,8 @@ cudaError_t launch_variant(const LinearLaunch& p, cudaStream_t s, int dev, int c
 
 }  // namespace
 
-void set_cluster_override(int g) { g_cluster_override = g; }
-void set_variant_override(int v) { g_variant_override = v; }
+void set_cluster_override(int g) { g_cluster_override.store(g, std::memory_order_relaxed); }
+void set_variant_override(int v) { g_variant_override.store(v, std::memory_order_relaxed); }
 
 cudaError_t launch_lora_linear(const LinearLaunch& p, cudaStream_t s, bool* driver_failed) {
   *driver_failed = false;
@@ -1024,8 +1026,8 @@ cudaError_t launch_lora_linear(const LinearLaunch& p, cudaStream_t s, bool* driv
   // single-SM panels for small K; above, SM pairs with 256 x 256 tiles, one
   // pair per panel up to K = 4096 and two beyond (clusters of 4: the panel's
   // x is fetched once for four SMs).
-  int variant = g_variant_override;
-  int cluster = g_cluster_override;
+  int variant = g_variant_override.load(std::memory_order_relaxed);
+  int cluster = g_cluster_override.load(std::memory_order_relaxed);
   if (variant == 0) {
     if (p.K <= 2048 || cluster == 1) {
       variant = 1;
