@@ -26,6 +26,9 @@ Sources (the pages are cited by title and section):
   Easy as 1, 2, 3", SC'11 (the pages name no generator).
 * Box-Muller: Box and Muller, "A Note on the Generation of Random Normal
   Deviates", Ann. Math. Statist. 29 (1958) (the pages only say eps ~ N(0, I)).
+* MXFP8: Open Compute Project, "OCP Microscaling Formats (MX) v1.0" and "OCP
+  8-bit Floating Point (OFP8)" (the pages only name MXFP8 linear layers,
+  section "Where the 3.9x speedup comes from" of the English article).
 
 Pins (tests/test_oracle_*.py, run with ``-m "not gpu"``):
 
@@ -40,8 +43,12 @@ Pins (tests/test_oracle_*.py, run with ``-m "not gpu"``):
                  to a plain GEMM, associativity through the dense merged
                  delta, merge identity B_cat A_cat = sum_i s_i B_i A_i and the
                  pages' 2.2e-8 merge-error figure.
+* mxfp8       -- the E4M3 bit layout, PyTorch's independent float8_e4m3fn
+                 conversion, round-to-nearest-even at every midpoint,
+                 saturation, the block-exponent definition, the 3-bit-mantissa
+                 error bound and brute-force loops on a tiny layer.
 
 Every function here has a pin; none is "parity unpinned".
 """
 
-from . import flow, lora, noise, philox  # noqa: F401
+from . import flow, lora, mxfp8, noise, philox  # noqa: F401
