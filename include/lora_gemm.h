@@ -192,6 +192,33 @@ lg_status lg_lora_linear_noalloc(const void* x, const void* W, const float* A_ca
                                  void* y, int64_t M, int K, int N, int R, void* stream);
 
 /* ------------------------------------------------------------------------
+ * lg_mx_quantize -- MXFP8 quantization of bf16 rows along K.  "Open-H3-
+ * Regenerate-2K: High-Resolution Video Refinement with Few-Step Diffusion",
+ * section "Where the 3.9x speedup comes from", runs the linear layers as MXFP8
+ * GEMMs with the activations re-quantized at every stage; the pages name the
+ * format only, so the block rule is the OCP Microscaling (MX) one:
+ *
+ *   blocks of 32 consecutive values along K share the scale 2^e with
+ *   e = floor(log2 max|v|) - 8 clamped to [-127, 127] (-127 for an all-zero
+ *   block), stored as the E8M0 byte e + 127; each value becomes the E4M3
+ *   (OCP E4M3FN) code of v 2^-e, round to nearest even, saturated at +-448.
+ *
+ *   in      DEVICE [rows, K] bf16 row-major.
+ *   codes   DEVICE [rows, K] uint8 row-major (E4M3 codes).
+ *   scales  DEVICE lg_mx_scale_bytes(rows, K) bytes of E8M0 scales, blocked:
+ *           rows in groups of 128, K in groups of 128 (four blocks); group
+ *           (g, kg) is 512 contiguous bytes at ((g * K / 128) + kg) * 512, the
+ *           byte of row r (0..127 in the group) and block b (0..3 in the K
+ *           group) at 16 (r mod 32) + 4 (r / 32) + b.  Rows past `rows`, up to
+ *           the next multiple of 128, get byte 0.
+ *
+ * Shapes: 0 <= rows < 2^31; K a multiple of 128.  in and codes 16-byte
+ * aligned; no buffer may overlap another.
+ * ---------------------------------------------------------------------- */
+size_t lg_mx_scale_bytes(int64_t rows, int K);
+lg_status lg_mx_quantize(const void* in, int64_t rows, int K, void* codes, void* scales, void* stream);
+
+/* ------------------------------------------------------------------------
  * lg_renoise -- partial re-noise of an upscaled latent:
  *
  *   x[i] = (1 - sigma) * up[i] + sigma * eps[offset + i],  i in [0, n)

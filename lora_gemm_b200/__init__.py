@@ -52,6 +52,8 @@ _SIGNATURES = {
         [_c_void_p, _c_void_p, _c_void_p, _c_void_p, _c_void_p, ctypes.c_int64, ctypes.c_int, ctypes.c_int,
          ctypes.c_int, _c_void_p],
     ),
+    "lg_mx_scale_bytes": (ctypes.c_size_t, [ctypes.c_int64, ctypes.c_int]),
+    "lg_mx_quantize": (ctypes.c_int, [_c_void_p, ctypes.c_int64, ctypes.c_int, _c_void_p, _c_void_p, _c_void_p]),
     "lg_renoise": (
         ctypes.c_int,
         [_c_void_p, _c_void_p, ctypes.c_int64, ctypes.c_float, ctypes.c_uint64, ctypes.c_uint64, _c_void_p],
@@ -219,6 +221,27 @@ def lora_linear(x, W, A_cat, B_cat, y=None, workspace=None):
                                 _ptr(workspace), ws_bytes, _stream(x.device))
     _check(st, "lg_lora_linear")
     return y
+
+
+def mx_scale_bytes(rows, K):
+    """Bytes of E8M0 scales lg_mx_quantize writes for [rows, K] (0 for an unsupported shape)."""
+    return int(lib.lg_mx_scale_bytes(int(rows), int(K)))
+
+
+def mx_quantize(x, codes=None, scales=None):
+    """MXFP8 of bf16 rows x [rows, K] along K: (E4M3 codes uint8 [rows, K],
+    E8M0 scales uint8 in the blocked layout of include/lora_gemm.h)."""
+    _need(x, torch.bfloat16, "x", 2)
+    rows, K = x.shape
+    if codes is None:
+        codes = torch.empty((rows, K), dtype=torch.uint8, device=x.device)
+    if scales is None:
+        scales = torch.empty(max(mx_scale_bytes(rows, K), 1), dtype=torch.uint8, device=x.device)
+    _need(codes, torch.uint8, "codes", 2)
+    with torch.cuda.device(x.device):
+        st = lib.lg_mx_quantize(_ptr(x), rows, K, _ptr(codes), _ptr(scales), _stream(x.device))
+    _check(st, "lg_mx_quantize")
+    return codes, scales
 
 
 def lora_linear_noalloc(x, W, A_cat, B_cat, y):

@@ -157,6 +157,29 @@ lg_status lg_lora_merge(int n_adapters, const float* const* A, const float* cons
   return launched(lg::launch_merge(pa, pb, A_cat, B_cat, sms, as_stream(stream)), 2);
 }
 
+size_t lg_mx_scale_bytes(int64_t rows, int K) {
+  if (rows < 0 || K < 128 || K % 128 || K > kMaxDim) return 0;
+  return (size_t)((rows + 127) / 128 * 128) * (size_t)(K / 32);
+}
+
+lg_status lg_mx_quantize(const void* in, int64_t rows, int K, void* codes, void* scales, void* stream) {
+  if (rows < 0 || K < 0) return LG_ERR_INVALID_ARG;
+  if (rows >= (int64_t)1 << 31 || K < 128 || K % 128 || K > kMaxDim) return LG_ERR_UNSUPPORTED_SHAPE;
+  if (!in || !codes || !scales) return LG_ERR_INVALID_ARG;
+  if (!aligned16(in) || !aligned16(codes)) return LG_ERR_MISALIGNED;
+  const uint64_t bi = 2ull * rows * K, bc = 1ull * rows * K, bs = lg_mx_scale_bytes(rows, K);
+  if (rows > 0 && (overlaps(in, bi, codes, bc) || overlaps(in, bi, scales, bs) || overlaps(codes, bc, scales, bs)))
+    return LG_ERR_INVALID_ARG;
+  if (rows == 0) return LG_OK;
+  int sms = 0;
+  lg_status st = current_device(&sms);
+  if (st != LG_OK) return st;
+  return launched(lg::launch_mx_quantize(reinterpret_cast<const uint16_t*>(in), rows, K,
+                                         reinterpret_cast<uint8_t*>(codes), reinterpret_cast<uint8_t*>(scales), sms,
+                                         as_stream(stream)),
+                  1);
+}
+
 size_t lg_lora_linear_workspace_size(int64_t M, int K, int N, int R) {
   if (M < 0 || K < 64 || N < 32 || K % 64 || N % 32 || K > kMaxDim || N > kMaxDim) return 0;
   if (R < 0 || R % 64 || R > kMaxRank) return 0;

@@ -41,6 +41,11 @@ cudaError_t launch_merge(const MergeAParams& pa, const MergeBParams& pb, float* 
 cudaError_t launch_prep_bf16(const float* A_cat, const float* B_cat, uint16_t* dstA, uint16_t* dstB,
                              int64_t nA, int64_t nB, int sm_count, cudaStream_t s);
 
+// MXFP8 quantization of bf16 rows [rows, K] along K (K % 128 == 0): E4M3
+// codes [rows, K] and E8M0 scales in the 128 x 128 blocked layout.
+cudaError_t launch_mx_quantize(const uint16_t* in, int64_t rows, int K, uint8_t* codes, uint8_t* scales,
+                               int sm_count, cudaStream_t s);
+
 // Merged-LoRA linear (tcgen05 kernel).  Factors already in bf16.
 struct LinearLaunch {
   const void* x;
