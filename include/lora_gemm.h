@@ -159,6 +159,31 @@ lg_status lg_lora_linear(const void* x, const void* W, const float* A_cat, const
                          void* workspace, size_t ws_bytes, void* stream);
 
 /* ------------------------------------------------------------------------
+ * lg_lora_linear_mxfp8 -- the merged-LoRA linear layer with the base term as
+ * MXFP8 GEMMs ("Open-H3-Regenerate-2K: High-Resolution Video Refinement with
+ * Few-Step Diffusion", section "Where the 3.9x speedup comes from"):
+ *
+ *   y = deq(x_codes, x_scales) deq(W_codes, W_scales)^T + (x A_cat^T) B_cat^T
+ *
+ * with deq the exact values of lg_mx_quantize's output (code value times the
+ * block's 2^e); the LoRA term is that of lg_lora_linear, from the bf16 x.
+ *
+ *   x                  DEVICE [M, K] bf16 (the activations x_codes came from).
+ *   x_codes, x_scales  DEVICE lg_mx_quantize(x) output ([M, K] codes,
+ *                      lg_mx_scale_bytes(M, K) scale bytes).
+ *   W_codes, W_scales  DEVICE lg_mx_quantize(W) output for W [N, K].
+ *   A_cat, B_cat, y, workspace, ws_bytes  as for lg_lora_linear.
+ *
+ * Arithmetic: tcgen05.mma kind::mxf8f6f4 with E8M0 block scales for the
+ * base term, FP32 accumulation; the LoRA term as in lg_lora_linear.
+ * Shapes: as lg_lora_linear, and K a multiple of 128.  All pointers 16-byte
+ * aligned; y must not overlap any input or the workspace.
+ * ---------------------------------------------------------------------- */
+lg_status lg_lora_linear_mxfp8(const void* x, const void* x_codes, const void* x_scales, const void* W_codes,
+                               const void* W_scales, const float* A_cat, const float* B_cat, void* y,
+                               int64_t M, int K, int N, int R, void* workspace, size_t ws_bytes, void* stream);
+
+/* ------------------------------------------------------------------------
  * lg_lora_linear_noalloc -- lg_lora_linear for callers that cannot allocate
  * device memory.  The pages have no counterpart; this is an interface
  * addition of this library.

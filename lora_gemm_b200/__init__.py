@@ -47,6 +47,11 @@ _SIGNATURES = {
         [_c_void_p, _c_void_p, _c_void_p, _c_void_p, _c_void_p, ctypes.c_int64, ctypes.c_int, ctypes.c_int,
          ctypes.c_int, _c_void_p, ctypes.c_size_t, _c_void_p],
     ),
+    "lg_lora_linear_mxfp8": (
+        ctypes.c_int,
+        [_c_void_p, _c_void_p, _c_void_p, _c_void_p, _c_void_p, _c_void_p, _c_void_p, _c_void_p, ctypes.c_int64,
+         ctypes.c_int, ctypes.c_int, ctypes.c_int, _c_void_p, ctypes.c_size_t, _c_void_p],
+    ),
     "lg_lora_linear_noalloc": (
         ctypes.c_int,
         [_c_void_p, _c_void_p, _c_void_p, _c_void_p, _c_void_p, ctypes.c_int64, ctypes.c_int, ctypes.c_int,
@@ -242,6 +247,44 @@ def mx_quantize(x, codes=None, scales=None):
         st = lib.lg_mx_quantize(_ptr(x), rows, K, _ptr(codes), _ptr(scales), _stream(x.device))
     _check(st, "lg_mx_quantize")
     return codes, scales
+
+
+def lora_linear_mxfp8(x, x_mx, W_mx, A_cat, B_cat, y=None, workspace=None):
+    """lora_linear with the base term as MXFP8 GEMMs: x_mx = mx_quantize(x),
+    W_mx = mx_quantize(W) (pairs of codes and scales); the LoRA term from the
+    bf16 x.  K must be a multiple of 128."""
+    _need(x, torch.bfloat16, "x", 2)
+    xq, xsf = x_mx
+    wq, wsf = W_mx
+    _need(xq, torch.uint8, "x codes", 2)
+    _need(wq, torch.uint8, "W codes", 2)
+    M, K = x.shape
+    N = wq.shape[0]
+    if tuple(xq.shape) != (M, K) or wq.shape[1] != K:
+        raise ValueError("codes must be [M, K] and [N, K]")
+    if xsf.numel() < mx_scale_bytes(M, K) or wsf.numel() < mx_scale_bytes(N, K):
+        raise ValueError("scale buffers too small")
+    R = 0
+    if A_cat is not None and A_cat.numel() > 0:
+        _need(A_cat, torch.float32, "A_cat", 2)
+        _need(B_cat, torch.float32, "B_cat", 2)
+        R = A_cat.shape[0]
+        if A_cat.shape[1] != K or tuple(B_cat.shape) != (N, R):
+            raise ValueError("A_cat must be [R, K] and B_cat [N, R]")
+    else:
+        A_cat = B_cat = None
+    if y is None:
+        y = torch.empty((M, N), dtype=torch.bfloat16, device=x.device)
+    _need(y, torch.bfloat16, "y", 2)
+    need = lora_linear_workspace_size(M, K, N, R)
+    if workspace is None and need > 0:
+        workspace = torch.empty(need, dtype=torch.uint8, device=x.device)
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    with torch.cuda.device(x.device):
+        st = lib.lg_lora_linear_mxfp8(_ptr(x), _ptr(xq), _ptr(xsf), _ptr(wq), _ptr(wsf), _ptr(A_cat), _ptr(B_cat),
+                                      _ptr(y), M, K, N, R, _ptr(workspace), ws_bytes, _stream(x.device))
+    _check(st, "lg_lora_linear_mxfp8")
+    return y
 
 
 def lora_linear_noalloc(x, W, A_cat, B_cat, y):

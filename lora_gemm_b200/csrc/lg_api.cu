@@ -187,15 +187,30 @@ size_t lg_lora_linear_workspace_size(int64_t M, int K, int N, int R) {
   return (size_t)(align256(2ull * R * K) + align256(2ull * N * R));
 }
 
-lg_status lg_lora_linear(const void* x, const void* W, const float* A_cat, const float* B_cat, void* y, int64_t M,
-                         int K, int N, int R, void* workspace, size_t ws_bytes, void* stream) {
+namespace {
+
+// MXFP8 operands of lg_lora_linear_mxfp8 (null for the bf16 layer).
+struct MxOperands {
+  const void* xq;
+  const void* xsf;
+  const void* wq;
+  const void* wsf;
+};
+
+lg_status lora_linear_impl(const void* x, const void* W, const float* A_cat, const float* B_cat, void* y, int64_t M,
+                           int K, int N, int R, void* workspace, size_t ws_bytes, void* stream,
+                           const MxOperands* mx) {
   if (M < 0 || K < 0 || N < 0 || R < 0) return LG_ERR_INVALID_ARG;
   if (M >= (int64_t)1 << 31 || K < 64 || N < 32 || K % 64 || N % 32 || K > kMaxDim || N > kMaxDim)
     return LG_ERR_UNSUPPORTED_SHAPE;
   if (R % 64 || R > kMaxRank) return LG_ERR_UNSUPPORTED_SHAPE;
-  if (!x || !W || !y) return LG_ERR_INVALID_ARG;
+  if (mx && K % 128) return LG_ERR_UNSUPPORTED_SHAPE;
+  if (!x || !y || (!mx && !W)) return LG_ERR_INVALID_ARG;
+  if (mx && (!mx->xq || !mx->xsf || !mx->wq || !mx->wsf)) return LG_ERR_INVALID_ARG;
   if (R > 0 && (!A_cat || !B_cat)) return LG_ERR_INVALID_ARG;
-  if (!aligned16(x) || !aligned16(W) || !aligned16(y)) return LG_ERR_MISALIGNED;
+  if (!aligned16(x) || !aligned16(y) || (!mx && !aligned16(W))) return LG_ERR_MISALIGNED;
+  if (mx && (!aligned16(mx->xq) || !aligned16(mx->xsf) || !aligned16(mx->wq) || !aligned16(mx->wsf)))
+    return LG_ERR_MISALIGNED;
   if (R > 0 && (!aligned16(A_cat) || !aligned16(B_cat))) return LG_ERR_MISALIGNED;
   const size_t need = lg_lora_linear_workspace_size(M, K, N, R);
   if (R > 0) {
@@ -204,13 +219,16 @@ lg_status lg_lora_linear(const void* x, const void* W, const float* A_cat, const
   }
   const uint64_t bx = 2ull * M * K, bw = 2ull * N * K, by = 2ull * M * N;
   if (M > 0) {
-    if (overlaps(y, by, x, bx) || overlaps(y, by, W, bw)) return LG_ERR_INVALID_ARG;
+    if (overlaps(y, by, x, bx) || (!mx && overlaps(y, by, W, bw))) return LG_ERR_INVALID_ARG;
+    if (mx && (overlaps(y, by, mx->xq, 1ull * M * K) || overlaps(y, by, mx->wq, 1ull * N * K) ||
+               overlaps(y, by, mx->xsf, lg_mx_scale_bytes(M, K)) || overlaps(y, by, mx->wsf, lg_mx_scale_bytes(N, K))))
+      return LG_ERR_INVALID_ARG;
     if (R > 0 && (overlaps(y, by, A_cat, 4ull * R * K) || overlaps(y, by, B_cat, 4ull * N * R) ||
                   overlaps(y, by, workspace, need)))
       return LG_ERR_INVALID_ARG;
   }
   if (R > 0 && (overlaps(workspace, need, A_cat, 4ull * R * K) || overlaps(workspace, need, B_cat, 4ull * N * R) ||
-                overlaps(workspace, need, x, bx) || overlaps(workspace, need, W, bw)))
+                overlaps(workspace, need, x, bx) || (!mx && overlaps(workspace, need, W, bw))))
     return LG_ERR_INVALID_ARG;
   if (M == 0) return LG_OK;
   int sms = 0;
@@ -237,10 +255,31 @@ lg_status lg_lora_linear(const void* x, const void* W, const float* A_cat, const
   p.R = R;
   p.sm_count = sms;
   p.wait_limit_ns = g_wait_limit_ns.load(std::memory_order_relaxed);
+  if (mx) {
+    p.mx = true;
+    p.xq = mx->xq;
+    p.xsf = mx->xsf;
+    p.wq = mx->wq;
+    p.wsf = mx->wsf;
+  }
   bool driver_failed = false;
   cudaError_t e = lg::launch_lora_linear(p, s, &driver_failed);
   if (e != cudaSuccess) cudaGetLastError();
   return launched(e, 1);
+}
+
+}  // namespace
+
+lg_status lg_lora_linear(const void* x, const void* W, const float* A_cat, const float* B_cat, void* y, int64_t M,
+                         int K, int N, int R, void* workspace, size_t ws_bytes, void* stream) {
+  return lora_linear_impl(x, W, A_cat, B_cat, y, M, K, N, R, workspace, ws_bytes, stream, nullptr);
+}
+
+lg_status lg_lora_linear_mxfp8(const void* x, const void* x_codes, const void* x_scales, const void* W_codes,
+                               const void* W_scales, const float* A_cat, const float* B_cat, void* y, int64_t M,
+                               int K, int N, int R, void* workspace, size_t ws_bytes, void* stream) {
+  const MxOperands mx{x_codes, x_scales, W_codes, W_scales};
+  return lora_linear_impl(x, nullptr, A_cat, B_cat, y, M, K, N, R, workspace, ws_bytes, stream, &mx);
 }
 
 lg_status lg_renoise(const float* up, float* x, int64_t n, float sigma, uint64_t seed, uint64_t offset,

@@ -460,6 +460,51 @@ __device__ __forceinline__ void umma_ts_pair(uint32_t d_tmem, uint32_t a_tmem, u
       "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
       : "memory");
 }
+// Block-scaled MXFP8 MMA (E4M3 A and B in shared memory, E8M0 scale factors
+// in tensor memory), SM pair: D[M=256, N] (+)= (A x sfa) (B x sfb)^T over
+// K = 32.  The scale-factor IDs (which byte of each 32-bit scale word) are
+// in the instruction descriptor.
+__device__ __forceinline__ void umma_mx_pair(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                             uint32_t sfa_tmem, uint32_t sfb_tmem, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::2.kind::mxf8f6f4.block_scale [%0], %1, %2, %3, [%5], [%6], p;\n\t}" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate), "r"(sfa_tmem), "r"(sfb_tmem)
+      : "memory");
+}
+
+// Instruction descriptor, kind::mxf8f6f4 with block scaling: E4M3 A and B
+// (both K-major), E8M0 scale factors, dense K = 32; sf_a / sf_b select the
+// byte of the 32-bit scale word each row's scale is taken from.
+__host__ __device__ constexpr uint32_t idesc_mx_e4m3(int m, int n, uint32_t sf_a, uint32_t sf_b) {
+  return (sf_b << 4)                      // B scale-factor ID
+         | (0u << 7) | (0u << 10)        // A, B format: E4M3
+         | ((uint32_t)(n >> 3) << 17)    // N / 8
+         | (1u << 23)                    // scale format: E8M0
+         | ((uint32_t)(m >> 4) << 24)    // M / 16
+         | (sf_a << 29);                 // A scale-factor ID
+}
+
+// Shared-memory descriptor of 32 rows of 16 bytes stored contiguously, no
+// swizzle (four 8-row core matrices 128 bytes apart): the source layout of a
+// tcgen05.cp 32x128b copy.
+__device__ __forceinline__ uint64_t plain_rows16_desc(uint32_t smem_addr) {
+  uint64_t d = 0;
+  d |= (uint64_t)((smem_addr & 0x3FFFFu) >> 4);
+  d |= (uint64_t)(128 >> 4) << 16;  // leading byte offset (one core matrix along the row)
+  d |= (uint64_t)(128 >> 4) << 32;  // stride byte offset: 128 B between 8-row core matrices
+  d |= (uint64_t)1 << 46;           // descriptor version for sm_100
+  return d;                          // layout type 0: no swizzle
+}
+
+// Shared -> tensor memory copy of 32 rows x 128 bits, replicated to all four
+// lane quarters (lanes 32 q + i, columns taddr .. +3 get row i), in both CTAs
+// of an SM pair.  Ordered with the issuing thread's later tcgen05.mma.
+__device__ __forceinline__ void tmem_cp_32x128b_x4_pair(uint32_t taddr, uint64_t sdesc) {
+  asm volatile("tcgen05.cp.cta_group::2.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sdesc) : "memory");
+}
+
 // Arrive once on the mbarrier at offset `bar` in every CTA of `cta_mask` when
 // all previously issued tcgen05 operations of this thread have completed.
 __device__ __forceinline__ void umma_commit_pair_mc(uint32_t bar, uint16_t cta_mask) {

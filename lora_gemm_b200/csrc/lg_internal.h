@@ -57,6 +57,14 @@ struct LinearLaunch {
   int K, N, R;
   int sm_count;
   uint64_t wait_limit_ns;
+  // MXFP8 base term (lg_lora_linear_mxfp8): E4M3 codes and blocked E8M0
+  // scales of x [M, K] and W [N, K]; x above stays the bf16 activations (the
+  // LoRA path reads them), W is unused.
+  bool mx = false;
+  const void* xq = nullptr;
+  const void* xsf = nullptr;
+  const void* wq = nullptr;
+  const void* wsf = nullptr;
 };
 // Returns cudaSuccess or the failing CUDA error; *driver_failed is set when
 // the tensor-map encoder (driver API) is missing or rejects a map.

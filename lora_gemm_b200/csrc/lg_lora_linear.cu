@@ -72,6 +72,8 @@ constexpr uint64_t TEARDOWN_LIMIT_NS = 200ull * 1000ull * 1000ull;
 constexpr size_t kMaxSmem = 232448;  // sm_100 opt-in maximum per block
 
 constexpr uint32_t H_TILE_BYTES = BM * BK * 2;  // 16 KiB: 64 ranks of h for 128 rows
+constexpr int BKQ = 128;                        // MXFP8: K elements per stage (128-byte rows)
+constexpr uint32_t SF_GROUP_BYTES = 512;         // MXFP8 scales of 128 rows x 128 K
 // Pair variant: y leaves through a TMA store, staged per epilogue warp in
 // 32 x 32 bf16 boxes (64-byte rows, 64-byte swizzle).
 constexpr int Y_BOX = 32;
@@ -87,23 +89,38 @@ constexpr uint32_t Y_STAGE_BYTES = 8 * Y_WARP_BYTES;              // 16 KiB for 
 // ranks [512, 576) live in a 16 KiB shared-memory tile (the up-projection
 // reads them from there as an ordinary shared-memory A operand), which costs
 // one stage of the ring but gives every stage 7 % more work per byte.
-template <bool PAIR>
+//
+// MX = true (pairs only): the base term x W^T runs as block-scaled MXFP8
+// MMAs (tcgen05.mma kind::mxf8f6f4, E4M3 operands, one E8M0 scale per 32
+// values along K) over stages of 128 K elements -- the same 16 KiB x and W
+// tiles, plus the scale groups (512 bytes per 128 rows): each CTA's own 128
+// x rows and all 256 W rows of the tile (the pair's MMA takes the B scales of
+// the whole N = 256 from each CTA's tensor memory), copied into tensor memory
+// (tcgen05.cp) before the stage's MMAs.  The scales take 32 TMEM columns (two
+// stages' worth of 4 + 8), so TMEM holds ranks [0, 448) of h and ranks
+// [448, 576) sit in two shared-memory tiles.
+template <bool PAIR, bool MX = false>
 struct Cfg {
-  static constexpr int BN = PAIR ? 256 : 224;               // output columns per tile
-  static constexpr uint32_t H_COL = (uint32_t)BN;            // first TMEM column of h
-  static constexpr int R_TMEM = (int)(TMEM_COLS - BN) * 2;  // ranks of h held in TMEM
-  static constexpr bool H_SMEM = R_TMEM < RMAX;              // the rest in shared memory
-  static constexpr int HALF_N = BN / 2;                      // accumulator columns per epilogue warp
-  static constexpr uint32_t B_ROWS = PAIR ? BN / 2 : BN;    // W / B_cat rows a CTA loads
-  static constexpr uint32_t B_BYTES = B_ROWS * BK * 2;
-  static constexpr uint32_t STAGE = A_BYTES + B_BYTES;
+  static constexpr int BN = PAIR ? 256 : 224;                         // output columns per tile
+  static constexpr uint32_t SF_COLS = MX ? 32u : 0u;                   // TMEM columns for MXFP8 scales
+  static constexpr uint32_t SF_COL = TMEM_COLS - SF_COLS;              // first of them
+  static constexpr uint32_t H_COL = (uint32_t)BN;                      // first TMEM column of h
+  static constexpr int R_TMEM = (int)(TMEM_COLS - BN - SF_COLS) * 2;  // ranks of h held in TMEM
+  static constexpr bool H_SMEM = R_TMEM < RMAX;                        // the rest in shared memory
+  static constexpr int H_TILES = (RMAX - R_TMEM + BK - 1) / BK;        // 16 KiB tiles of 64 ranks
+  static constexpr int HALF_N = BN / 2;                                // accumulator columns per epilogue warp
+  static constexpr uint32_t B_ROWS = PAIR ? BN / 2 : BN;              // W / B_cat rows a CTA loads
+  static constexpr uint32_t B_BYTES = B_ROWS * BK * 2;                // also 128 rows x 128 E4M3 codes
+  static constexpr uint32_t SF_OFF = A_BYTES + B_BYTES;               // MX: x scales, then 2 groups of W scales
+  static constexpr uint32_t STAGE = A_BYTES + B_BYTES + (MX ? 2048u : 0u);
   static constexpr int MMA_M = PAIR ? 2 * BM : BM;
   static constexpr int PANEL = PAIR ? 2 * BM : BM;
+  static_assert(!MX || PAIR, "the MXFP8 base term runs on SM pairs only");
   static_assert(STAGE % 1024 == 0, "stages must stay 1024-byte aligned");
   static_assert((PAIR ? HC_MAX / 2 : HC_MAX) * BK * 2 <= B_BYTES, "A_cat chunk tile must fit the B slot");
-  static_assert(RMAX - R_TMEM <= BK, "ranks beyond TMEM must fit one shared-memory K block");
   static_assert(R_TMEM % BK == 0, "the TMEM / shared-memory split of h must fall on a K block");
   static_assert(HALF_N % 16 == 0 && HC_MAX <= BN, "epilogue and chunk widths");
+  static_assert(SF_COL + SF_COLS == TMEM_COLS && SF_OFF + (MX ? 2048u : 0u) == STAGE, "TMEM and stage layout");
 };
 
 struct Control {
@@ -127,6 +144,7 @@ struct Args {
   int num_panels;
   int n_tiles;
   int k_blocks;
+  int kq_blocks;  // MXFP8: stages of 128 K elements in the base-term loop
   int r_blocks;
   int group;        // members (CTAs, or pairs) sharing one panel
   int slice;        // ranks of h each member computes (R when group == 1)
@@ -210,11 +228,12 @@ __device__ __forceinline__ void chunk_ranks(const Args& a, int member, int j, in
 // x tiles loaded last are the first ones the next sweep of the same panel
 // re-reads, while they are still in L2.
 // ---------------------------------------------------------------------------
-template <bool PAIR>
+template <bool PAIR, bool MX>
 __device__ void run_producer(const CUtensorMap* tm_x, const CUtensorMap* tm_w, const CUtensorMap* tm_a,
-                             const CUtensorMap* tm_b, const Args& a, Control* ctl, uint32_t smem_base,
+                             const CUtensorMap* tm_b, const CUtensorMap* tm_xq, const CUtensorMap* tm_sfa,
+                             const CUtensorMap* tm_sfb, const Args& a, Control* ctl, uint32_t smem_base,
                              uint32_t crank, uint32_t cid, uint32_t ncl, volatile int* abort_flag) {
-  using C = Cfg<PAIR>;
+  using C = Cfg<PAIR, MX>;
   const uint32_t stages = (uint32_t)a.stages;
   const int member = PAIR ? (int)(crank >> 1) : (int)crank;
   const int half = PAIR ? (int)(crank & 1) : 0;
@@ -226,7 +245,7 @@ __device__ void run_producer(const CUtensorMap* tm_x, const CUtensorMap* tm_w, c
   const uint32_t a_rows = PAIR ? (uint32_t)a.chunk_n / 2 : (uint32_t)a.chunk_n;
   const uint32_t mult = PAIR ? 2u : 1u;
   const uint32_t tx_a = mult * (A_BYTES + a_rows * BK * 2);
-  const uint32_t tx_k = mult * C::STAGE;
+  const uint32_t tx_k = mult * (A_BYTES + C::B_BYTES + (MX ? 3 * SF_GROUP_BYTES : 0u));
   const uint32_t tx_r = mult * C::B_BYTES;
   uint32_t stage = 0, phase = 0, sweep = 0, it = 0;
   uint64_t fills = 0;
@@ -241,11 +260,11 @@ __device__ void run_producer(const CUtensorMap* tm_x, const CUtensorMap* tm_w, c
   // x panels are re-read once per N tile: keep them in L2 ahead of the
   // streamed weight tiles.
   const uint64_t pol_x = l2_policy_evict_last();
-  auto load_x = [&](uint32_t dst, int c0, int c1) {
+  auto load_x = [&](const CUtensorMap* m, uint32_t dst, int c0, int c1) {
     if constexpr (PAIR) {
-      tma_load_2d_pair_hint(dst, tm_x, full0 + 8 * stage, c0, c1, pol_x);
+      tma_load_2d_pair_hint(dst, m, full0 + 8 * stage, c0, c1, pol_x);
     } else {
-      tma_load_2d_hint(dst, tm_x, full0 + 8 * stage, c0, c1, pol_x);
+      tma_load_2d_hint(dst, m, full0 + 8 * stage, c0, c1, pol_x);
     }
   };
   for (int p = (int)cid; ok && p < a.num_panels; p += (int)ncl, ++it) {
@@ -261,7 +280,7 @@ __device__ void run_producer(const CUtensorMap* tm_x, const CUtensorMap* tm_w, c
         }
         const uint32_t sa = smem_base + stage * C::STAGE;
         if (posts_tx) mbar_arrive_expect_tx(full_local + 8 * stage, tx_a);
-        load_x(sa, kb * BK, m0);
+        load_x(tm_x, sa, kb * BK, m0);
         load(tm_a, sa + A_BYTES, kb * BK, first + half * (int)a_rows);
         ++fills;
         advance(stage, phase, stages);
@@ -276,16 +295,29 @@ __device__ void run_producer(const CUtensorMap* tm_x, const CUtensorMap* tm_w, c
     }
     for (int t = member; ok && t < a.n_tiles; t += a.group, ++sweep) {
       const int n0 = t * C::BN + half * (int)C::B_ROWS;
-      for (int i = 0; i < a.k_blocks; ++i) {
-        const int kb = (sweep & 1) ? a.k_blocks - 1 - i : i;
+      const int kloop = MX ? a.kq_blocks : a.k_blocks;
+      for (int i = 0; i < kloop; ++i) {
+        const int kb = (sweep & 1) ? kloop - 1 - i : i;
         if (!wait_bounded(empty0 + 8 * stage, phase ^ 1, a.wait_limit_ns, abort_flag)) {
           ok = false;
           break;
         }
         const uint32_t sa = smem_base + stage * C::STAGE;
         if (posts_tx) mbar_arrive_expect_tx(full_local + 8 * stage, tx_k);
-        load_x(sa, kb * BK, m0);
-        load(tm_w, sa + A_BYTES, kb * BK, n0);
+        if constexpr (MX) {
+          // E4M3 codes of x and W (128 K per stage), the scale group of this
+          // CTA's x rows and both groups of the tile's 256 W rows: group
+          // (row block, K block) is two 256-byte rows of the scale map.
+          const int nb = t * C::BN / BM;
+          load_x(tm_xq, sa, kb * BKQ, m0);
+          load(tm_w, sa + A_BYTES, kb * BKQ, n0);
+          load(tm_sfa, sa + C::SF_OFF, 0, 2 * ((m0 / BM) * a.kq_blocks + kb));
+          load(tm_sfb, sa + C::SF_OFF + SF_GROUP_BYTES, 0, 2 * (nb * a.kq_blocks + kb));
+          load(tm_sfb, sa + C::SF_OFF + 2 * SF_GROUP_BYTES, 0, 2 * ((nb + 1) * a.kq_blocks + kb));
+        } else {
+          load_x(tm_x, sa, kb * BK, m0);
+          load(tm_w, sa + A_BYTES, kb * BK, n0);
+        }
         ++fills;
         advance(stage, phase, stages);
       }
@@ -321,14 +353,14 @@ __device__ void run_producer(const CUtensorMap* tm_x, const CUtensorMap* tm_w, c
 // ---------------------------------------------------------------------------
 // MMA issuer (warp 1, one thread; for pairs only the leader).
 // ---------------------------------------------------------------------------
-template <bool PAIR>
+template <bool PAIR, bool MX>
 __device__ void run_mma(const Args& a, Control* ctl, uint32_t smem_base, uint32_t tmem, uint32_t crank, uint32_t cid,
                         uint32_t ncl, volatile int* abort_flag) {
-  using C = Cfg<PAIR>;
+  using C = Cfg<PAIR, MX>;
   const uint32_t stages = (uint32_t)a.stages;
   const int member = PAIR ? (int)(crank >> 1) : (int)crank;
   const uint16_t mask = (uint16_t)(3u << (2 * member));
-  uint32_t stage = 0, phase = 0, acc_phase = 0;
+  uint32_t stage = 0, phase = 0, acc_phase = 0, sf_buf = 0;
   bool ok = true;
   const uint32_t full0 = smem_u32(&ctl->full[0]);
   const uint32_t empty0 = smem_u32(&ctl->empty[0]);
@@ -389,7 +421,8 @@ __device__ void run_mma(const Args& a, Control* ctl, uint32_t smem_base, uint32_
         break;
       }
       tc_fence_after();
-      for (int i = 0; i < a.k_blocks; ++i) {
+      const int kloop = MX ? a.kq_blocks : a.k_blocks;
+      for (int i = 0; i < kloop; ++i) {
         if (!wait_bounded(full0 + 8 * stage, phase, a.wait_limit_ns, abort_flag)) {
           ok = false;
           break;
@@ -398,8 +431,26 @@ __device__ void run_mma(const Args& a, Control* ctl, uint32_t smem_base, uint32_
         const uint32_t sa = smem_base + stage * C::STAGE;
         const uint64_t da = sw128_kmajor_desc(sa);
         const uint64_t db = sw128_kmajor_desc(sa + A_BYTES);
+        if constexpr (MX) {
+          // This stage's scales into one of two TMEM scale buffers (x rows in
+          // columns +0..3, W rows 0-127 in +4..7 and 128-255 in +8..11: row
+          // n's word sits in column n / 32), then four K = 32 MMAs, the k-th
+          // taking byte k of each row's scale word.  tcgen05.cp and
+          // tcgen05.mma of this thread run in issue order.
+          const uint32_t sf = tmem + C::SF_COL + 16u * (sf_buf & 1u);
+          ++sf_buf;
+          tmem_cp_32x128b_x4_pair(sf, plain_rows16_desc(sa + C::SF_OFF));
+          tmem_cp_32x128b_x4_pair(sf + 4, plain_rows16_desc(sa + C::SF_OFF + SF_GROUP_BYTES));
+          tmem_cp_32x128b_x4_pair(sf + 8, plain_rows16_desc(sa + C::SF_OFF + 2 * SF_GROUP_BYTES));
 #pragma unroll
-        for (int kk = 0; kk < BK / 16; ++kk) mma_ss(da + 2 * kk, db + 2 * kk, idesc_y, (i | kk) != 0);
+          for (int kk = 0; kk < BKQ / 32; ++kk) {
+            umma_mx_pair(d_acc, da + 2 * kk, db + 2 * kk, idesc_mx_e4m3(C::MMA_M, C::BN, (uint32_t)kk, (uint32_t)kk),
+                         sf, sf + 4, (i | kk) != 0);
+          }
+        } else {
+#pragma unroll
+          for (int kk = 0; kk < BK / 16; ++kk) mma_ss(da + 2 * kk, db + 2 * kk, idesc_y, (i | kk) != 0);
+        }
         commit(empty0 + 8 * stage);
         advance(stage, phase, stages);
       }
@@ -418,8 +469,9 @@ __device__ void run_mma(const Args& a, Control* ctl, uint32_t smem_base, uint32_
             mma_ts(tmem + C::H_COL + (uint32_t)(rb * (BK / 2) + kk * 8), db + 2 * kk);
           }
         } else {
-          // The last 64 ranks of h: A from the shared-memory tile.
-          const uint64_t dh = sw128_kmajor_desc(smem_base + a.h_tile_off);
+          // Ranks past R_TMEM: A from the shared-memory tiles of h.
+          const uint64_t dh =
+              sw128_kmajor_desc(smem_base + a.h_tile_off + (uint32_t)(rb * BK - C::R_TMEM) / BK * H_TILE_BYTES);
 #pragma unroll
           for (int kk = 0; kk < BK / 16; ++kk) mma_ss(dh + 2 * kk, db + 2 * kk, idesc_y, 1u);
         }
@@ -449,13 +501,13 @@ __device__ void run_mma(const Args& a, Control* ctl, uint32_t smem_base, uint32_
 // ---------------------------------------------------------------------------
 struct HRow {
   uint32_t lane_base;  // TMEM address of this warp's lane quarter
-  uint32_t tile_row;   // shared address of this thread's row of the h tile
+  uint32_t tile_row;   // shared address of this thread's row of the first h tile (16 KiB apart)
   uint32_t sw;         // row mod 8
 };
 
-template <bool PAIR, int WORDS>
+template <bool PAIR, bool MX, int WORDS>
 __device__ __forceinline__ void h_put(const HRow& h, int r0, const uint32_t (&v)[WORDS]) {
-  using C = Cfg<PAIR>;
+  using C = Cfg<PAIR, MX>;
   if (!C::H_SMEM || r0 < C::R_TMEM) {
     if constexpr (WORDS == 8) {
       tmem_st_32x32b_x8(h.lane_base + C::H_COL + (uint32_t)(r0 / 2), v);
@@ -463,15 +515,17 @@ __device__ __forceinline__ void h_put(const HRow& h, int r0, const uint32_t (&v)
       tmem_st_32x32b_x4(h.lane_base + C::H_COL + (uint32_t)(r0 / 2), v);
     }
   } else {
-    const uint32_t c = (uint32_t)(r0 - C::R_TMEM) / 8;
-    st_shared_v4(h.tile_row + ((c ^ h.sw) << 4), v[0], v[1], v[2], v[3]);
-    if constexpr (WORDS == 8) st_shared_v4(h.tile_row + (((c + 1) ^ h.sw) << 4), v[4], v[5], v[6], v[7]);
+    const uint32_t k = (uint32_t)(r0 - C::R_TMEM);
+    const uint32_t row = h.tile_row + k / BK * H_TILE_BYTES;
+    const uint32_t c = (k % BK) / 8;
+    st_shared_v4(row + ((c ^ h.sw) << 4), v[0], v[1], v[2], v[3]);
+    if constexpr (WORDS == 8) st_shared_v4(row + (((c + 1) ^ h.sw) << 4), v[4], v[5], v[6], v[7]);
   }
 }
 
-template <bool PAIR, int WORDS>
+template <bool PAIR, bool MX, int WORDS>
 __device__ __forceinline__ void h_get(const HRow& h, int r0, uint32_t (&v)[WORDS]) {
-  using C = Cfg<PAIR>;
+  using C = Cfg<PAIR, MX>;
   if (!C::H_SMEM || r0 < C::R_TMEM) {
     if constexpr (WORDS == 8) {
       tmem_ld_32x32b_x8(h.lane_base + C::H_COL + (uint32_t)(r0 / 2), v);
@@ -480,15 +534,17 @@ __device__ __forceinline__ void h_get(const HRow& h, int r0, uint32_t (&v)[WORDS
     }
     tmem_wait_ld();
   } else {
-    const uint32_t c = (uint32_t)(r0 - C::R_TMEM) / 8;
-    ld_shared_v4(h.tile_row + ((c ^ h.sw) << 4), v[0], v[1], v[2], v[3]);
-    if constexpr (WORDS == 8) ld_shared_v4(h.tile_row + (((c + 1) ^ h.sw) << 4), v[4], v[5], v[6], v[7]);
+    const uint32_t k = (uint32_t)(r0 - C::R_TMEM);
+    const uint32_t row = h.tile_row + k / BK * H_TILE_BYTES;
+    const uint32_t c = (k % BK) / 8;
+    ld_shared_v4(row + ((c ^ h.sw) << 4), v[0], v[1], v[2], v[3]);
+    if constexpr (WORDS == 8) ld_shared_v4(row + (((c + 1) ^ h.sw) << 4), v[4], v[5], v[6], v[7]);
   }
 }
 
 // FP32 accumulator columns [0, count) = ranks first .. first+count-1 -> bf16
 // pairs in h.  count is a multiple of 8.
-template <bool PAIR>
+template <bool PAIR, bool MX>
 __device__ __forceinline__ void acc_to_h(const HRow& h, int first, int count, int half) {
   const int full_blocks = count / 16;
   for (int b = half; b < full_blocks; b += 2) {
@@ -498,7 +554,7 @@ __device__ __forceinline__ void acc_to_h(const HRow& h, int first, int count, in
     uint32_t packed[8];
 #pragma unroll
     for (int i = 0; i < 8; ++i) packed[i] = pack_bf16x2(__uint_as_float(v[2 * i]), __uint_as_float(v[2 * i + 1]));
-    h_put<PAIR, 8>(h, first + 16 * b, packed);
+    h_put<PAIR, MX, 8>(h, first + 16 * b, packed);
   }
   if ((count % 16) && ((full_blocks & 1) == half)) {
     uint32_t v[8];
@@ -507,42 +563,42 @@ __device__ __forceinline__ void acc_to_h(const HRow& h, int first, int count, in
     uint32_t packed[4];
 #pragma unroll
     for (int i = 0; i < 4; ++i) packed[i] = pack_bf16x2(__uint_as_float(v[2 * i]), __uint_as_float(v[2 * i + 1]));
-    h_put<PAIR, 4>(h, first + 16 * full_blocks, packed);
+    h_put<PAIR, MX, 4>(h, first + 16 * full_blocks, packed);
   }
   tmem_wait_st();
 }
 
 // This member's slice of h (ranks s0 .. s0 + slice - 1) into its staging row.
-template <bool PAIR>
+template <bool PAIR, bool MX>
 __device__ __forceinline__ void h_to_staging(const HRow& h, int s0, int slice, int half, uint32_t row) {
   const int blocks = slice / 16;
   for (int b = half; b < blocks; b += 2) {
     uint32_t v[8];
-    h_get<PAIR, 8>(h, s0 + 16 * b, v);
+    h_get<PAIR, MX, 8>(h, s0 + 16 * b, v);
     st_shared_v4(row + 32u * b, v[0], v[1], v[2], v[3]);
     st_shared_v4(row + 32u * b + 16, v[4], v[5], v[6], v[7]);
   }
   if ((slice % 16) && ((blocks & 1) == half)) {
     uint32_t v[4];
-    h_get<PAIR, 4>(h, s0 + 16 * blocks, v);
+    h_get<PAIR, MX, 4>(h, s0 + 16 * blocks, v);
     st_shared_v4(row + 32u * blocks, v[0], v[1], v[2], v[3]);
   }
 }
 
 // A peer's staged slice (cluster address of its row) into this CTA's h.
-template <bool PAIR>
+template <bool PAIR, bool MX>
 __device__ __forceinline__ void staging_to_h(const HRow& h, int s0, int slice, int half, uint32_t remote_row) {
   const int blocks = slice / 16;
   for (int b = half; b < blocks; b += 2) {
     uint32_t v[8];
     ld_shared_cluster_v4(remote_row + 32u * b, v[0], v[1], v[2], v[3]);
     ld_shared_cluster_v4(remote_row + 32u * b + 16, v[4], v[5], v[6], v[7]);
-    h_put<PAIR, 8>(h, s0 + 16 * b, v);
+    h_put<PAIR, MX, 8>(h, s0 + 16 * b, v);
   }
   if ((slice % 16) && ((blocks & 1) == half)) {
     uint32_t v[4];
     ld_shared_cluster_v4(remote_row + 32u * blocks, v[0], v[1], v[2], v[3]);
-    h_put<PAIR, 4>(h, s0 + 16 * blocks, v);
+    h_put<PAIR, MX, 4>(h, s0 + 16 * blocks, v);
   }
 }
 
@@ -550,10 +606,10 @@ __device__ __forceinline__ void staging_to_h(const HRow& h, int s0, int slice, i
 // Epilogue (warps 2..9): warp w reads TMEM lanes 32 (w mod 4) .. +31 and
 // handles half (w - 2) / 4 of the columns.
 // ---------------------------------------------------------------------------
-template <bool PAIR>
+template <bool PAIR, bool MX>
 __device__ void run_epilogue(const CUtensorMap* tm_y, const Args& a, Control* ctl, uint32_t smem_base, uint32_t tmem, uint32_t crank,
                              uint32_t cid, uint32_t ncl, int warp, int lane, volatile int* abort_flag) {
-  using C = Cfg<PAIR>;
+  using C = Cfg<PAIR, MX>;
   const int q = warp & 3;
   const int half = (warp - 2) >> 2;
   const int parity = PAIR ? (int)(crank & 1) : 0;
@@ -608,7 +664,7 @@ __device__ void run_epilogue(const CUtensorMap* tm_y, const Args& a, Control* ct
       tc_fence_after();
       int first, count;
       chunk_ranks(a, member, j, first, count);
-      acc_to_h<PAIR>(hr, first, count, half);
+      acc_to_h<PAIR, MX>(hr, first, count, half);
       if (a.group > 1 && j == a.n_chunks - 1) {
         // Swap slices with the other members of the group: stage this slice
         // at the start of the (idle) ring, wait for every member's, copy the
@@ -622,7 +678,7 @@ __device__ void run_epilogue(const CUtensorMap* tm_y, const Args& a, Control* ct
         if (!ok) break;
         tc_fence_after();
         fence_proxy_async_smem();
-        h_to_staging<PAIR>(hr, member * a.slice, a.slice, half, my_row);
+        h_to_staging<PAIR, MX>(hr, member * a.slice, a.slice, half, my_row);
         __syncwarp();
         if (lane == 0) {
           for (int c = 0; c < a.group; ++c) mbar_arrive_remote(mapa_shared(slice_ready, peer_rank(c)));
@@ -630,7 +686,7 @@ __device__ void run_epilogue(const CUtensorMap* tm_y, const Args& a, Control* ct
         ok = __all_sync(0xffffffffu, wait_bounded(slice_ready, it & 1, a.wait_limit_ns, abort_flag, true));
         if (!ok) break;
         for (int c = 0; c < a.group; ++c) {
-          if (c != member) staging_to_h<PAIR>(hr, c * a.slice, a.slice, half, mapa_shared(my_row, peer_rank(c)));
+          if (c != member) staging_to_h<PAIR, MX>(hr, c * a.slice, a.slice, half, mapa_shared(my_row, peer_rank(c)));
         }
         tmem_wait_st();
         __syncwarp();
@@ -709,11 +765,13 @@ __device__ void run_epilogue(const CUtensorMap* tm_y, const Args& a, Control* ct
   __syncwarp();
 }
 
-template <bool PAIR>
+template <bool PAIR, bool MX>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     k_lora_linear(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_w,
                   const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b,
-                  const __grid_constant__ CUtensorMap tm_y, const Args args) {
+                  const __grid_constant__ CUtensorMap tm_y, const __grid_constant__ CUtensorMap tm_xq,
+                  const __grid_constant__ CUtensorMap tm_sfa, const __grid_constant__ CUtensorMap tm_sfb,
+                  const Args args) {
   extern __shared__ uint8_t smem_raw[];
   // Dynamic shared memory starts at the same offset in every CTA, so after
   // rounding up to 1 KiB the layout (and every mapa'd address) matches.
@@ -743,6 +801,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     tma_prefetch_desc(&tm_x);
     tma_prefetch_desc(&tm_w);
     if (PAIR) tma_prefetch_desc(&tm_y);
+    if (MX) {
+      tma_prefetch_desc(&tm_xq);
+      tma_prefetch_desc(&tm_sfa);
+      tma_prefetch_desc(&tm_sfb);
+    }
     if (args.R > 0) {
       tma_prefetch_desc(&tm_a);
       tma_prefetch_desc(&tm_b);
@@ -765,13 +828,16 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   volatile int* abort_flag = &ctl->abort_flag;
 
   if (warp == 0) {
-    if (lane == 0) run_producer<PAIR>(&tm_x, &tm_w, &tm_a, &tm_b, args, ctl, smem_base, crank, cid, ncl, abort_flag);
+    if (lane == 0) {
+      run_producer<PAIR, MX>(&tm_x, &tm_w, &tm_a, &tm_b, &tm_xq, &tm_sfa, &tm_sfb, args, ctl, smem_base, crank, cid,
+                             ncl, abort_flag);
+    }
     __syncwarp();
   } else if (warp == 1) {
-    if (lane == 0 && issues_mma) run_mma<PAIR>(args, ctl, smem_base, tmem, crank, cid, ncl, abort_flag);
+    if (lane == 0 && issues_mma) run_mma<PAIR, MX>(args, ctl, smem_base, tmem, crank, cid, ncl, abort_flag);
     __syncwarp();
   } else {
-    run_epilogue<PAIR>(&tm_y, args, ctl, smem_base, tmem, crank, cid, ncl, warp, lane, abort_flag);
+    run_epilogue<PAIR, MX>(&tm_y, args, ctl, smem_base, tmem, crank, cid, ncl, warp, lane, abort_flag);
   }
 
   tc_fence_before();
@@ -825,6 +891,32 @@ bool make_map(PFN_cuTensorMapEncodeTiled_v12000 enc, CUtensorMap* m, const void*
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// Row-major E4M3 codes [outer, inner] read as tiles of box_outer rows x 128
+// codes with the 128-byte swizzle (the layout of the bf16 tiles above).
+bool make_map_codes(PFN_cuTensorMapEncodeTiled_v12000 enc, CUtensorMap* m, const void* base, uint64_t inner,
+                    uint64_t outer, uint32_t box_outer) {
+  cuuint64_t dims[2] = {inner, outer};
+  cuuint64_t strides[1] = {inner};
+  cuuint32_t box[2] = {(cuuint32_t)BKQ, box_outer};
+  cuuint32_t elem_strides[2] = {1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, elem_strides,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// MXFP8 scales (the blocked layout of lg_mx_quantize) viewed as rows of 256
+// bytes: a 512-byte group is a box of two rows.  Groups past the end read as
+// zero.
+bool make_map_scales(PFN_cuTensorMapEncodeTiled_v12000 enc, CUtensorMap* m, const void* base, uint64_t groups) {
+  cuuint64_t dims[2] = {256, groups * 2};
+  cuuint64_t strides[1] = {256};
+  cuuint32_t box[2] = {256, 2};
+  cuuint32_t elem_strides[2] = {1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, elem_strides,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 // Row-major bf16 y [rows, cols] written in 32 x 32 boxes from 64-byte-swizzled
 // shared memory; the store clips rows and columns outside the matrix.
 bool make_store_map(PFN_cuTensorMapEncodeTiled_v12000 enc, CUtensorMap* m, void* base, uint64_t cols,
@@ -847,9 +939,9 @@ struct Geometry {
   size_t smem = 0;
 };
 
-template <bool PAIR>
+template <bool PAIR, bool MX>
 bool make_geometry(int group, int R, Geometry* g) {
-  using C = Cfg<PAIR>;
+  using C = Cfg<PAIR, MX>;
   g->group = group;
   if (R > 0) {
     if (R % group) return false;
@@ -864,7 +956,7 @@ bool make_geometry(int group, int R, Geometry* g) {
     // one side of the split (slices and chunks start on multiples of 16).
     if (C::H_SMEM && R > C::R_TMEM && (g->slice % 16 || g->chunk_valid % 16)) return false;
   }
-  const uint32_t h_tile = C::H_SMEM ? H_TILE_BYTES : 0u;
+  const uint32_t h_tile = (uint32_t)C::H_TILES * H_TILE_BYTES;
   const uint32_t y_stage = PAIR ? Y_STAGE_BYTES : 0u;
   const size_t fixed = 1024 + h_tile + y_stage + sizeof(Control);
   g->stages = (int)((kMaxSmem - fixed) / C::STAGE);
@@ -889,7 +981,7 @@ int max_active_clusters(const void* kernel, int variant, int dev, int cluster, s
     bool known = false;
     int n = 0;
   };
-  static Entry cache[64][2][17];
+  static Entry cache[64][3][17];
   std::lock_guard<std::mutex> lock(mu);
   Entry* en = (dev >= 0 && dev < 64 && cluster <= 16) ? &cache[dev][variant - 1][cluster] : nullptr;
   if (en && en->known) return en->n;
@@ -921,7 +1013,8 @@ cudaError_t configure_kernels(int dev) {
   static bool configured[64] = {};
   std::lock_guard<std::mutex> lock(mu);
   if (dev >= 0 && dev < 64 && configured[dev]) return cudaSuccess;
-  const void* kernels[2] = {(const void*)k_lora_linear<false>, (const void*)k_lora_linear<true>};
+  const void* kernels[3] = {(const void*)k_lora_linear<false, false>, (const void*)k_lora_linear<true, false>,
+                            (const void*)k_lora_linear<true, true>};
   for (const void* k : kernels) {
     cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kMaxSmem);
     if (e == cudaSuccess) e = cudaFuncSetAttribute(k, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
@@ -931,17 +1024,29 @@ cudaError_t configure_kernels(int dev) {
   return cudaSuccess;
 }
 
-template <bool PAIR>
+template <bool PAIR, bool MX>
 cudaError_t launch_variant(const LinearLaunch& p, cudaStream_t s, int dev, int cluster, bool* driver_failed,
                            PFN_cuTensorMapEncodeTiled_v12000 enc) {
-  using C = Cfg<PAIR>;
+  using C = Cfg<PAIR, MX>;
   const int group = PAIR ? cluster / 2 : cluster;
   Geometry geo;
-  if (!make_geometry<PAIR>(group, p.R, &geo)) return cudaErrorInvalidConfiguration;
+  if (!make_geometry<PAIR, MX>(group, p.R, &geo)) return cudaErrorInvalidConfiguration;
   const uint32_t a_rows = PAIR ? (uint32_t)geo.chunk_n / 2 : (uint32_t)geo.chunk_n;
-  CUtensorMap tm_x, tm_w, tm_a, tm_b, tm_y;
-  bool ok = make_map(enc, &tm_x, p.x, (uint64_t)p.K, (uint64_t)p.M, BM) &&
-            make_map(enc, &tm_w, p.W, (uint64_t)p.K, (uint64_t)p.N, C::B_ROWS);
+  CUtensorMap tm_x, tm_w, tm_a, tm_b, tm_y, tm_xq, tm_sfa, tm_sfb;
+  bool ok = make_map(enc, &tm_x, p.x, (uint64_t)p.K, (uint64_t)p.M, BM);
+  if (MX) {
+    // Base term from the E4M3 codes and scales; phase A still reads bf16 x.
+    const uint64_t kg = (uint64_t)(p.K / BKQ);
+    ok = ok && make_map_codes(enc, &tm_w, p.wq, (uint64_t)p.K, (uint64_t)p.N, C::B_ROWS) &&
+         make_map_codes(enc, &tm_xq, p.xq, (uint64_t)p.K, (uint64_t)p.M, BM) &&
+         make_map_scales(enc, &tm_sfa, p.xsf, (uint64_t)((p.M + BM - 1) / BM) * kg) &&
+         make_map_scales(enc, &tm_sfb, p.wsf, (uint64_t)((p.N + BM - 1) / BM) * kg);
+  } else {
+    ok = ok && make_map(enc, &tm_w, p.W, (uint64_t)p.K, (uint64_t)p.N, C::B_ROWS);
+    tm_xq = tm_x;  // never read without MXFP8
+    tm_sfa = tm_x;
+    tm_sfb = tm_x;
+  }
   if (ok) {
     if (PAIR) {
       ok = make_store_map(enc, &tm_y, p.y, (uint64_t)p.N, (uint64_t)p.M);
@@ -968,6 +1073,7 @@ cudaError_t launch_variant(const LinearLaunch& p, cudaStream_t s, int dev, int c
   args.num_panels = (int)((p.M + C::PANEL - 1) / C::PANEL);
   args.n_tiles = (p.N + C::BN - 1) / C::BN;
   args.k_blocks = p.K / BK;
+  args.kq_blocks = MX ? p.K / BKQ : 0;
   args.r_blocks = p.R / BK;
   args.group = group;
   args.slice = geo.slice;
@@ -980,8 +1086,8 @@ cudaError_t launch_variant(const LinearLaunch& p, cudaStream_t s, int dev, int c
   args.h_tile_off = geo.h_tile_off;
   args.y_stage_off = geo.y_stage_off;
   args.wait_limit_ns = p.wait_limit_ns;
-  const void* kernel = (const void*)k_lora_linear<PAIR>;
-  int clusters = max_active_clusters(kernel, PAIR ? 2 : 1, dev, cluster, geo.smem, p.sm_count);
+  const void* kernel = (const void*)k_lora_linear<PAIR, MX>;
+  int clusters = max_active_clusters(kernel, MX ? 3 : (PAIR ? 2 : 1), dev, cluster, geo.smem, p.sm_count);
   if (clusters <= 0) clusters = p.sm_count / cluster;
   if (clusters > args.num_panels) clusters = args.num_panels;
   if (clusters < 1) clusters = 1;
@@ -998,7 +1104,7 @@ cudaError_t launch_variant(const LinearLaunch& p, cudaStream_t s, int dev, int c
   attr[0].val.clusterDim.z = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  void* params[6] = {&tm_x, &tm_w, &tm_a, &tm_b, &tm_y, &args};
+  void* params[9] = {&tm_x, &tm_w, &tm_a, &tm_b, &tm_y, &tm_xq, &tm_sfa, &tm_sfb, &args};
   cudaError_t e = cudaLaunchKernelExC(&cfg, kernel, params);
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
@@ -1037,14 +1143,22 @@ cudaError_t launch_lora_linear(const LinearLaunch& p, cudaStream_t s, bool* driv
       if (cluster == 0) cluster = p.K <= 4096 ? 2 : 4;
     }
   }
+  if (p.mx) {
+    // The MXFP8 base term runs on SM pairs only.
+    if (g_variant_override.load(std::memory_order_relaxed) == 0 && g_cluster_override.load(std::memory_order_relaxed) == 0)
+      cluster = p.K <= 4096 ? 2 : 4;
+    if (cluster < 2) cluster = 2;
+    if (cluster > 8) cluster = 8;
+    return launch_variant<true, true>(p, s, dev, cluster, driver_failed, enc);
+  }
   if (variant == 1) {
     if (cluster == 0) cluster = p.K <= 2048 ? 1 : 2;
     if (cluster > 8) cluster = 8;
-    return launch_variant<false>(p, s, dev, cluster, driver_failed, enc);
+    return launch_variant<false, false>(p, s, dev, cluster, driver_failed, enc);
   }
   if (cluster < 2) cluster = 2;
   if (cluster > 8) cluster = 8;
-  return launch_variant<true>(p, s, dev, cluster, driver_failed, enc);
+  return launch_variant<true, false>(p, s, dev, cluster, driver_failed, enc);
 }
 
 cudaError_t read_and_clear_device_error(cudaStream_t s, int* value) {
