@@ -217,6 +217,88 @@ def run_step(P, ev=None):
         rec(f"euler{k}", lambda k=k: lg.euler_step(P.x_lat, P.v[k], P.sigmas[k], P.sigmas[k + 1]))
 
 
+def run_mxfp8(P, args, world, peaks):
+    """The same step with the linear layers as MXFP8 GEMMs (lg_lora_linear_mxfp8):
+    W is quantized once (model load), each distinct x once per step inside
+    the timed region (it comes from the previous op in a real forward), the
+    LoRA path stays bf16.  Reported beside the bf16 headline, not instead of it."""
+    import lora_gemm_b200 as lg
+
+    wq = [lg.mx_quantize(L["W"]) for L in P.layers]
+    xq = {}
+    for L in P.layers:
+        if id(L["x"]) not in xq:
+            xq[id(L["x"])] = lg.mx_quantize(L["x"])
+    first_use = {}
+    for k, L in enumerate(P.layers):
+        first_use.setdefault(id(L["x"]), k)
+
+    def step(ev=None):
+        def rec(name, fn):
+            if ev is None:
+                fn()
+                return
+            s = torch.cuda.Event(enable_timing=True)
+            e = torch.cuda.Event(enable_timing=True)
+            s.record()
+            fn()
+            e.record()
+            ev.append((name, s, e))
+
+        for L in P.layers:
+            rec("lora_merge", lambda L=L: lg.lora_merge(L["As"], L["Bs"], P.scales, L["A_cat"], L["B_cat"]))
+        rec("renoise", lambda: lg.renoise(P.up, P.sigmas[0], P.w.seed, offset=P.noise_offset, out=P.x_lat))
+        for k, L in enumerate(P.layers):
+            if first_use[id(L["x"])] == k:
+                q = xq[id(L["x"])]
+                rec("quantize", lambda L=L, q=q: lg.mx_quantize(L["x"], codes=q[0], scales=q[1]))
+            rec(f"lin{k}", lambda k=k, L=L: lg.lora_linear_mxfp8(L["x"], xq[id(L["x"])], wq[k], L["A_cat"], L["B_cat"],
+                                                                  y=L["y"], workspace=L["ws"]))
+            rec(f"euler{k}", lambda k=k: lg.euler_step(P.x_lat, P.v[k], P.sigmas[k], P.sigmas[k + 1]))
+
+    for _ in range(max(args.warmup, 1)):
+        step()
+    torch.cuda.synchronize()
+    ev = []
+    barrier(world)
+    torch.cuda.synchronize()
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    t0.record()
+    for _ in range(args.steps):
+        step(ev)
+    t1.record()
+    torch.cuda.synchronize()
+    barrier(world)
+    status = lg.get_last_device_error()
+    if status != lg.LG_OK:
+        raise SystemExit(f"device error during the MXFP8 steps: {lg.status_string(status)}")
+    ms = max_over_ranks(t0.elapsed_time(t1), world)
+    per = {}
+    for name, s, e in ev:
+        per.setdefault(name, []).append(s.elapsed_time(e))
+    flops = [layer_flops(P.M, L["K"], L["N"], P.R) for L in P.layers]
+    lin_ms = [statistics.mean(per[f"lin{k}"]) for k in range(len(P.layers))]
+    tflops = sum(flops) / (sum(lin_ms) * 1e-3) / 1e12
+    fp8_peak = 2.0 * peaks["bf16_tflops_sustained"]
+    q_ms = sum(per["quantize"]) / args.steps
+    del xq, wq
+    return {
+        "value": round(_dist().whole_job_rate(P.M, world, args.steps, ms), 1), "unit": UNIT,
+        "ms_per_step": round(ms / args.steps, 3),
+        "lora_linear_mxfp8": {
+            "per_layer_ms": [round(t, 4) for t in lin_ms],
+            "per_layer_tflops": [round(f / (t * 1e-3) / 1e12, 1) for f, t in zip(flops, lin_ms)],
+            "tflops": round(tflops, 1),
+            "peak": round(fp8_peak, 1),
+            "peak_kind": "fp8 dense, derived: measured bf16 sustained x 2 (the nominal fp8 / bf16 ratio)",
+            "frac": round(tflops / fp8_peak, 4),
+        },
+        "quantize_x_ms_per_step": round(q_ms, 4),
+        "note": "W quantized once outside the timed steps; x quantized inside; LoRA path bf16",
+    }
+
+
 def bytes_per_kernel(P):
     w = P.w
     n = w.latent_numel
@@ -350,6 +432,8 @@ def run_ours(args, rank, world, local):
         "gpu_launches": int(launches),
         "launches_per_step": int(launches) // max(args.steps, 1),
     }
+    if not args.no_mxfp8:
+        result["mxfp8"] = run_mxfp8(P, args, world, peaks)
     if not args.no_e2e:
         result["e2e"] = run_e2e(P, args, world)
     if rank == 0 and not args.no_cpu_baseline:
@@ -627,6 +711,7 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default=WORKLOAD)
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-mxfp8", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--tokens", type=int, default=None,
