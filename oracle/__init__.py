@@ -46,7 +46,8 @@ Pins (tests/test_oracle_*.py, run with ``-m "not gpu"``):
 * mxfp8       -- the E4M3 bit layout, PyTorch's independent float8_e4m3fn
                  conversion, round-to-nearest-even at every midpoint,
                  saturation, the block-exponent definition, the 3-bit-mantissa
-                 error bound and brute-force loops on a tiny layer.
+                 error bound and brute-force loops on a tiny layer; SiLU
+                 against PyTorch's and its limits, SwiGLU by brute force.
 
 Every function here has a pin; none is "parity unpinned".
 """

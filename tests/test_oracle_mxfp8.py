@@ -147,3 +147,30 @@ def test_linear_close_to_unquantized_and_rank_zero():
     y0 = mx.lora_linear_mxfp8(x, W, np.zeros((0, K)), np.zeros((N, 0)))
     assert np.allclose(y0, mx.mx_dequantize(*mx.mx_quantize(x)) @ mx.mx_dequantize(*mx.mx_quantize(W)).T, rtol=0,
                        atol=1e-12)
+
+
+def test_silu_against_torch_and_limits():
+    g = np.concatenate([np.linspace(-30, 30, 2001), [0.0, 800.0, -800.0, 1e-300]])
+    ours = mx.silu(g)
+    ref = torch.nn.functional.silu(torch.from_numpy(g)).numpy()
+    assert np.allclose(ours, ref, rtol=1e-14, atol=1e-300)
+    assert mx.silu(0.0) == 0.0
+    assert mx.silu(800.0) == 800.0
+    assert mx.silu(-800.0) == 0.0
+
+
+def test_swiglu_brute_force_tiny():
+    rng = np.random.default_rng(21)
+    M, K, F, R = 3, 64, 32, 4
+    x = rng.standard_normal((M, K))
+    W2 = rng.standard_normal((2 * F, K)) * 0.2
+    A = rng.standard_normal((R, K)) * 0.1
+    B = rng.standard_normal((2 * F, R)) * 0.1
+    s, (codes, exps) = mx.swiglu_mxfp8(x, W2, A, B)
+    z = mx.lora_linear_mxfp8(x, W2, A, B)
+    for m in range(M):
+        for j in range(F):
+            g, u = z[m, j], z[m, F + j]
+            assert abs(s[m, j] - g / (1.0 + math.exp(-g)) * u) <= 1e-14 * (1 + abs(s[m, j]))
+    c2, e2 = mx.mx_quantize_scalar(s)
+    assert np.array_equal(codes, c2) and np.array_equal(exps, e2)
