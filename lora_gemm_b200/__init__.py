@@ -52,6 +52,11 @@ _SIGNATURES = {
         [_c_void_p, _c_void_p, _c_void_p, _c_void_p, _c_void_p, _c_void_p, _c_void_p, _c_void_p, ctypes.c_int64,
          ctypes.c_int, ctypes.c_int, ctypes.c_int, _c_void_p, ctypes.c_size_t, _c_void_p],
     ),
+    "lg_lora_linear_swiglu_mxfp8": (
+        ctypes.c_int,
+        [_c_void_p, _c_void_p, _c_void_p, _c_void_p, _c_void_p, _c_void_p, _c_void_p, _c_void_p, _c_void_p,
+         ctypes.c_int64, ctypes.c_int, ctypes.c_int, ctypes.c_int, _c_void_p, ctypes.c_size_t, _c_void_p],
+    ),
     "lg_lora_linear_noalloc": (
         ctypes.c_int,
         [_c_void_p, _c_void_p, _c_void_p, _c_void_p, _c_void_p, ctypes.c_int64, ctypes.c_int, ctypes.c_int,
@@ -285,6 +290,40 @@ def lora_linear_mxfp8(x, x_mx, W_mx, A_cat, B_cat, y=None, workspace=None):
                                       _ptr(y), M, K, N, R, _ptr(workspace), ws_bytes, _stream(x.device))
     _check(st, "lg_lora_linear_mxfp8")
     return y
+
+
+def lora_linear_swiglu_mxfp8(x, x_mx, W2_mx, A_cat, B_cat, out=None, workspace=None):
+    """MLP input projection with SwiGLU and the MXFP8 quantizer fused: W2 [2F, K]
+    (gate rows, then up rows) as mx_quantize(W2); returns (codes [M, F], scales)
+    of silu(z[:, :F]) * z[:, F:] with z = x W2^T + LoRA."""
+    _need(x, torch.bfloat16, "x", 2)
+    xq, xsf = x_mx
+    wq, wsf = W2_mx
+    M, K = x.shape
+    N2 = wq.shape[0]
+    F = N2 // 2
+    R = 0
+    if A_cat is not None and A_cat.numel() > 0:
+        _need(A_cat, torch.float32, "A_cat", 2)
+        _need(B_cat, torch.float32, "B_cat", 2)
+        R = A_cat.shape[0]
+        if A_cat.shape[1] != K or tuple(B_cat.shape) != (N2, R):
+            raise ValueError("A_cat must be [R, K] and B_cat [2F, R]")
+    else:
+        A_cat = B_cat = None
+    if out is None:
+        out = (torch.empty((M, F), dtype=torch.uint8, device=x.device),
+               torch.empty(max(mx_scale_bytes(M, F), 1), dtype=torch.uint8, device=x.device))
+    need = lora_linear_workspace_size(M, K, N2, R)
+    if workspace is None and need > 0:
+        workspace = torch.empty(need, dtype=torch.uint8, device=x.device)
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    with torch.cuda.device(x.device):
+        st = lib.lg_lora_linear_swiglu_mxfp8(_ptr(x), _ptr(xq), _ptr(xsf), _ptr(wq), _ptr(wsf), _ptr(A_cat),
+                                             _ptr(B_cat), _ptr(out[0]), _ptr(out[1]), M, K, F, R, _ptr(workspace),
+                                             ws_bytes, _stream(x.device))
+    _check(st, "lg_lora_linear_swiglu_mxfp8")
+    return out
 
 
 def lora_linear_noalloc(x, W, A_cat, B_cat, y):

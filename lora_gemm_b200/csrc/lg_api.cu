@@ -197,18 +197,29 @@ struct MxOperands {
   const void* wsf;
 };
 
+// Fused SwiGLU output of lg_lora_linear_swiglu_mxfp8 (null otherwise).
+struct SwigluOut {
+  void* codes;
+  void* scales;
+};
+
 lg_status lora_linear_impl(const void* x, const void* W, const float* A_cat, const float* B_cat, void* y, int64_t M,
                            int K, int N, int R, void* workspace, size_t ws_bytes, void* stream,
-                           const MxOperands* mx) {
+                           const MxOperands* mx, const SwigluOut* sw = nullptr) {
   if (M < 0 || K < 0 || N < 0 || R < 0) return LG_ERR_INVALID_ARG;
   if (M >= (int64_t)1 << 31 || K < 64 || N < 32 || K % 64 || N % 32 || K > kMaxDim || N > kMaxDim)
     return LG_ERR_UNSUPPORTED_SHAPE;
   if (R % 64 || R > kMaxRank) return LG_ERR_UNSUPPORTED_SHAPE;
   if (mx && K % 128) return LG_ERR_UNSUPPORTED_SHAPE;
-  if (!x || !y || (!mx && !W)) return LG_ERR_INVALID_ARG;
+  if (sw && (!mx || N % 256)) return LG_ERR_UNSUPPORTED_SHAPE;
+  if (sw) {
+    if (!sw->codes || !sw->scales) return LG_ERR_INVALID_ARG;
+    if (!aligned16(sw->codes) || !aligned16(sw->scales)) return LG_ERR_MISALIGNED;
+  }
+  if (!x || (!sw && !y) || (!mx && !W)) return LG_ERR_INVALID_ARG;
   if (mx && (!mx->xq || !mx->xsf || !mx->wq || !mx->wsf)) return LG_ERR_INVALID_ARG;
   if (R > 0 && (!A_cat || !B_cat)) return LG_ERR_INVALID_ARG;
-  if (!aligned16(x) || !aligned16(y) || (!mx && !aligned16(W))) return LG_ERR_MISALIGNED;
+  if (!aligned16(x) || (!sw && !aligned16(y)) || (!mx && !aligned16(W))) return LG_ERR_MISALIGNED;
   if (mx && (!aligned16(mx->xq) || !aligned16(mx->xsf) || !aligned16(mx->wq) || !aligned16(mx->wsf)))
     return LG_ERR_MISALIGNED;
   if (R > 0 && (!aligned16(A_cat) || !aligned16(B_cat))) return LG_ERR_MISALIGNED;
@@ -217,7 +228,18 @@ lg_status lora_linear_impl(const void* x, const void* W, const float* A_cat, con
     if (!workspace || ws_bytes < need) return LG_ERR_WORKSPACE;
     if (!aligned16(workspace)) return LG_ERR_MISALIGNED;
   }
-  const uint64_t bx = 2ull * M * K, bw = 2ull * N * K, by = 2ull * M * N;
+  const uint64_t bx = 2ull * M * K, bw = 2ull * N * K;
+  // The output region: y, or the SwiGLU codes and scales.
+  const void* out = sw ? sw->codes : y;
+  const uint64_t by = sw ? 1ull * M * (N / 2) : 2ull * M * N;
+  if (sw && M > 0) {
+    const uint64_t bs = lg_mx_scale_bytes(M, N / 2);
+    if (overlaps(sw->codes, by, sw->scales, bs) || overlaps(sw->scales, bs, x, bx) ||
+        overlaps(sw->scales, bs, mx->xq, 1ull * M * K) || overlaps(sw->scales, bs, mx->wq, 1ull * N * K) ||
+        (R > 0 && overlaps(sw->scales, bs, workspace, need)))
+      return LG_ERR_INVALID_ARG;
+  }
+  y = const_cast<void*>(out);
   if (M > 0) {
     if (overlaps(y, by, x, bx) || (!mx && overlaps(y, by, W, bw))) return LG_ERR_INVALID_ARG;
     if (mx && (overlaps(y, by, mx->xq, 1ull * M * K) || overlaps(y, by, mx->wq, 1ull * N * K) ||
@@ -262,6 +284,12 @@ lg_status lora_linear_impl(const void* x, const void* W, const float* A_cat, con
     p.wq = mx->wq;
     p.wsf = mx->wsf;
   }
+  if (sw) {
+    p.y = nullptr;
+    p.ffn = N / 2;
+    p.q_codes = sw->codes;
+    p.q_scales = sw->scales;
+  }
   bool driver_failed = false;
   cudaError_t e = lg::launch_lora_linear(p, s, &driver_failed);
   if (e != cudaSuccess) cudaGetLastError();
@@ -280,6 +308,17 @@ lg_status lg_lora_linear_mxfp8(const void* x, const void* x_codes, const void* x
                                int K, int N, int R, void* workspace, size_t ws_bytes, void* stream) {
   const MxOperands mx{x_codes, x_scales, W_codes, W_scales};
   return lora_linear_impl(x, nullptr, A_cat, B_cat, y, M, K, N, R, workspace, ws_bytes, stream, &mx);
+}
+
+lg_status lg_lora_linear_swiglu_mxfp8(const void* x, const void* x_codes, const void* x_scales, const void* W_codes,
+                                      const void* W_scales, const float* A_cat, const float* B_cat, void* out_codes,
+                                      void* out_scales, int64_t M, int K, int F, int R, void* workspace,
+                                      size_t ws_bytes, void* stream) {
+  if (F < 0 || F > kMaxDim / 2) return LG_ERR_UNSUPPORTED_SHAPE;
+  if (F % 128) return LG_ERR_UNSUPPORTED_SHAPE;
+  const MxOperands mx{x_codes, x_scales, W_codes, W_scales};
+  const SwigluOut sw{out_codes, out_scales};
+  return lora_linear_impl(x, nullptr, A_cat, B_cat, nullptr, M, K, 2 * F, R, workspace, ws_bytes, stream, &mx, &sw);
 }
 
 lg_status lg_renoise(const float* up, float* x, int64_t n, float sigma, uint64_t seed, uint64_t offset,

@@ -65,6 +65,11 @@ struct LinearLaunch {
   const void* xsf = nullptr;
   const void* wq = nullptr;
   const void* wsf = nullptr;
+  // Fused SwiGLU (MXFP8 only): N = 2 ffn (gate rows, then up rows); the
+  // MXFP8 codes [M, ffn] and blocked scales of silu(gate) * up replace y.
+  int ffn = 0;
+  void* q_codes = nullptr;
+  void* q_scales = nullptr;
 };
 // Returns cudaSuccess or the failing CUDA error; *driver_failed is set when
 // the tensor-map encoder (driver API) is missing or rejects a map.

@@ -46,6 +46,7 @@
 #include <cstdlib>
 #include <mutex>
 
+#include <cuda_fp8.h>
 #include <cudaTypedefs.h>
 
 #include "../../include/lora_gemm.h"
@@ -156,6 +157,13 @@ struct Args {
   uint32_t control_off;     // byte offset of the Control block
   uint32_t h_tile_off;      // byte offset of the shared-memory tile of h (pair variant)
   uint32_t y_stage_off;     // byte offset of the y staging boxes (pair variant)
+  // SwiGLU + MXFP8 output (MX variant, ffn > 0): W holds ffn gate rows then
+  // ffn up rows; tile t covers gate rows [128 t, 128 t + 128) (leader CTA of
+  // the pair) and the matching up rows (follower), and the epilogue writes
+  // the MXFP8 codes and scales of silu(gate) * up instead of y.
+  int ffn;
+  uint8_t* q_codes;   // [M, ffn]
+  uint8_t* q_scales;  // blocked layout, ffn / 128 K groups
   unsigned long long wait_limit_ns;
 };
 
@@ -294,7 +302,7 @@ __device__ void run_producer(const CUtensorMap* tm_x, const CUtensorMap* tm_w, c
       fence_proxy_async_smem();
     }
     for (int t = member; ok && t < a.n_tiles; t += a.group, ++sweep) {
-      const int n0 = t * C::BN + half * (int)C::B_ROWS;
+      const int n0 = a.ffn > 0 ? (half ? a.ffn : 0) + t * BM : t * C::BN + half * (int)C::B_ROWS;
       const int kloop = MX ? a.kq_blocks : a.k_blocks;
       for (int i = 0; i < kloop; ++i) {
         const int kb = (sweep & 1) ? kloop - 1 - i : i;
@@ -308,12 +316,13 @@ __device__ void run_producer(const CUtensorMap* tm_x, const CUtensorMap* tm_w, c
           // E4M3 codes of x and W (128 K per stage), the scale group of this
           // CTA's x rows and both groups of the tile's 256 W rows: group
           // (row block, K block) is two 256-byte rows of the scale map.
-          const int nb = t * C::BN / BM;
+          const int nb0 = a.ffn > 0 ? t : t * C::BN / BM;                 // row block of B rows 0-127
+          const int nb1 = a.ffn > 0 ? a.ffn / BM + t : t * C::BN / BM + 1;  // ... and of rows 128-255
           load_x(tm_xq, sa, kb * BKQ, m0);
           load(tm_w, sa + A_BYTES, kb * BKQ, n0);
           load(tm_sfa, sa + C::SF_OFF, 0, 2 * ((m0 / BM) * a.kq_blocks + kb));
-          load(tm_sfb, sa + C::SF_OFF + SF_GROUP_BYTES, 0, 2 * (nb * a.kq_blocks + kb));
-          load(tm_sfb, sa + C::SF_OFF + 2 * SF_GROUP_BYTES, 0, 2 * ((nb + 1) * a.kq_blocks + kb));
+          load(tm_sfb, sa + C::SF_OFF + SF_GROUP_BYTES, 0, 2 * (nb0 * a.kq_blocks + kb));
+          load(tm_sfb, sa + C::SF_OFF + 2 * SF_GROUP_BYTES, 0, 2 * (nb1 * a.kq_blocks + kb));
         } else {
           load_x(tm_x, sa, kb * BK, m0);
           load(tm_w, sa + A_BYTES, kb * BK, n0);
@@ -602,6 +611,57 @@ __device__ __forceinline__ void staging_to_h(const HRow& h, int s0, int slice, i
   }
 }
 
+// Fused SwiGLU + MXFP8 quantizer for one token row: s = silu(g) * u over 64
+// consecutive output columns (col0 .. col0 + 63, two blocks of 32), each block
+// quantized by the MX rule (scale 2^e, e = floor(log2 max|s|) - 8 clamped to
+// [-127, 127], -127 for an all-zero block; E4M3 codes of s 2^-e, round to
+// nearest even, saturated) -- the same rule as lg_mx_quantize, applied to the
+// FP32 products.  Rows past the matrix up to the next multiple of 128 get
+// scale byte 0 (the blocked scale layout covers them).
+__device__ __forceinline__ void swiglu_quantize_store(const Args& a, int64_t row, int col0, const uint32_t (&g)[2][32],
+                                                      const uint32_t (&u)[2][32]) {
+  if (row >= (a.M + 127) / 128 * 128) return;
+  const int k_groups = a.ffn / 128;
+  const int64_t grp = row >> 7;
+  const int r = (int)(row & 127);
+  for (int b = 0; b < 2; ++b) {
+    const int kb = col0 / 32 + b;
+    uint8_t* sf = a.q_scales + (((grp * k_groups + (kb >> 2)) << 9) + 16 * (r & 31) + 4 * (r >> 5) + (kb & 3));
+    if (row >= a.M) {
+      *sf = 0;
+      continue;
+    }
+    float v[32];
+    float amax = 0.f;
+#pragma unroll
+    for (int i = 0; i < 32; ++i) {
+      const float gv = __uint_as_float(g[b][i]);
+      v[i] = gv / (1.0f + expf(-gv)) * __uint_as_float(u[b][i]);
+      amax = fmaxf(amax, fabsf(v[i]));
+    }
+    int e = -127;
+    if (amax > 0.f) {
+      int ex;
+      frexpf(amax, &ex);
+      e = min(max(ex - 1 - 8, -127), 127);
+    }
+    const float inv = e == 127 ? __uint_as_float(0x00400000u) : __uint_as_float((uint32_t)(127 - e) << 23);
+    uint32_t out[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const __nv_fp8x2_storage_t lo =
+          __nv_cvt_float2_to_fp8x2(make_float2(v[4 * i] * inv, v[4 * i + 1] * inv), __NV_SATFINITE, __NV_E4M3);
+      const __nv_fp8x2_storage_t hi =
+          __nv_cvt_float2_to_fp8x2(make_float2(v[4 * i + 2] * inv, v[4 * i + 3] * inv), __NV_SATFINITE, __NV_E4M3);
+      out[i] = (uint32_t)lo | ((uint32_t)hi << 16);
+    }
+    uint4* dst = reinterpret_cast<uint4*>(a.q_codes + row * (int64_t)a.ffn + col0 + 32 * b);
+    dst[0] = make_uint4(out[0], out[1], out[2], out[3]);
+    dst[1] = make_uint4(out[4], out[5], out[6], out[7]);
+    *sf = (uint8_t)(e + 127);
+  }
+}
+
 // ---------------------------------------------------------------------------
 // Epilogue (warps 2..9): warp w reads TMEM lanes 32 (w mod 4) .. +31 and
 // handles half (w - 2) / 4 of the columns.
@@ -700,6 +760,22 @@ __device__ void run_epilogue(const CUtensorMap* tm_y, const Args& a, Control* ct
       ok = __all_sync(0xffffffffu, wait_bounded(acc_full, acc_phase, a.wait_limit_ns, abort_flag));
       if (!ok) break;
       tc_fence_after();
+      if constexpr (MX) {
+        if (a.ffn > 0) {
+          // Fused SwiGLU: accumulator columns [0, 128) are gate rows and
+          // [128, 256) the matching up rows; this warp takes 64 of each.
+          uint32_t g[2][32], u[2][32];
+          const uint32_t gsrc = lane_base + ACC_COL + (uint32_t)(64 * half);
+          tmem_ld_32x32b_x32(gsrc, g[0]);
+          tmem_ld_32x32b_x32(gsrc + 32, g[1]);
+          tmem_ld_32x32b_x32(gsrc + 128, u[0]);
+          tmem_ld_32x32b_x32(gsrc + 160, u[1]);
+          tmem_wait_ld();
+          release_acc(false);
+          swiglu_quantize_store(a, m0 + row_in_tile, t * BM + 64 * half, g, u);
+          continue;
+        }
+      }
       // Pull this warp's HALF_N accumulator columns into registers and hand
       // the accumulator back at once, so the next tile's MMAs overlap the
       // conversion and the stores below.
@@ -1048,10 +1124,10 @@ cudaError_t launch_variant(const LinearLaunch& p, cudaStream_t s, int dev, int c
     tm_sfb = tm_x;
   }
   if (ok) {
-    if (PAIR) {
+    if (PAIR && p.ffn == 0) {
       ok = make_store_map(enc, &tm_y, p.y, (uint64_t)p.N, (uint64_t)p.M);
     } else {
-      tm_y = tm_x;  // never used: the single-SM epilogue stores directly
+      tm_y = tm_x;  // never used: the single-SM epilogue stores directly, SwiGLU writes MXFP8
     }
   }
   if (ok && p.R > 0) {
@@ -1071,7 +1147,10 @@ cudaError_t launch_variant(const LinearLaunch& p, cudaStream_t s, int dev, int c
   args.N = p.N;
   args.R = p.R;
   args.num_panels = (int)((p.M + C::PANEL - 1) / C::PANEL);
-  args.n_tiles = (p.N + C::BN - 1) / C::BN;
+  args.n_tiles = p.ffn > 0 ? p.ffn / BM : (p.N + C::BN - 1) / C::BN;
+  args.ffn = p.ffn;
+  args.q_codes = reinterpret_cast<uint8_t*>(p.q_codes);
+  args.q_scales = reinterpret_cast<uint8_t*>(p.q_scales);
   args.k_blocks = p.K / BK;
   args.kq_blocks = MX ? p.K / BKQ : 0;
   args.r_blocks = p.R / BK;
