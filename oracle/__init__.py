@@ -38,7 +38,10 @@ Pins (tests/test_oracle_*.py, run with ``-m "not gpu"``):
                  special words (u1 = 1, u2 = 0, u2 = 1/4), distribution tests.
 * flow        -- exact recovery of z0 along the linear flow path with the
                  exact velocity; sigma = 0 / 1 special cases; Sterbenz
-                 exactness of the schedule coefficients in FP32.
+                 exactness of the schedule coefficients in FP32; the
+                 projection with the Euler update by brute-force loops over
+                 the latent's flat index and by exact recovery of z0 with
+                 x = I (a wrong token-to-cell map misses).
 * lora        -- brute-force pure-Python loops on tiny shapes, rank 0 reduces
                  to a plain GEMM, associativity through the dense merged
                  delta, merge identity B_cat A_cat = sum_i s_i B_i A_i and the

@@ -35,6 +35,8 @@ FP64 from those exact inputs.
 
 import numpy as np
 
+from oracle import lora
+
 # Printed schedule, "Three steps instead of dozens".
 SCHEDULE_DECIMAL = (0.909, 0.857, 0.667, 0.0)
 # IC starts, "三步接着放大的草稿画，八步从噪声重画".
@@ -69,6 +71,26 @@ def euler_step(x, v, sigma, sigma_next):
     x = np.asarray(x, dtype=np.float64)
     v = np.asarray(v, dtype=np.float64)
     return x + (float(sigma_next) - float(sigma)) * v
+
+
+def projection_euler_step(x, W, A_cat, B_cat, z, frame_tokens, sigma, sigma_next):
+    """The step's last projection followed by its Euler update (FP64).
+
+    The projection v = lora.lora_linear(x, W, A_cat, B_cat) [M, C] gives each
+    token its C velocity channels.  Token m is cell p = m mod T of frame
+    f = m div T (T = frame_tokens, the H W cells of a frame); the latent z
+    keeps the [F, C, H W] layout, so v[f T + p, c] is the velocity of
+    z[f, c, p].  Returns euler_step(z, that velocity, sigma, sigma_next) with
+    z's shape.  The pages fold nothing here; this is the plain composition of
+    the layer ("The four-stage refinement pipeline") and the update ("Three
+    steps instead of dozens").
+    """
+    v = lora.lora_linear(x, W, A_cat, B_cat)
+    M, C = v.shape
+    T = int(frame_tokens)
+    v_latent = v.reshape(M // T, T, C).transpose(0, 2, 1)
+    z = np.asarray(z, np.float64)
+    return euler_step(z.reshape(M // T, C, T), v_latent, sigma, sigma_next).reshape(z.shape)
 
 
 def flow_point(z0, eps, sigma):

@@ -156,3 +156,56 @@ def test_reference_row_blend():
     up = np.array([1.0, -2.0, 0.0])
     eps = np.array([0.0, 1.0, 5.0])
     np.testing.assert_array_equal(flow.renoise(up, eps, sig), (1 - sig) * up + sig * eps)
+
+
+def test_projection_euler_brute_force_tiny():
+    """The fused projection + Euler oracle against explicit loops over the
+    latent's flat index ((f C + c) T + p), with a rank-2 LoRA."""
+    rng = np.random.default_rng(31)
+    F, C, T, K, R = 2, 3, 5, 8, 2
+    M = F * T
+    x = rng.standard_normal((M, K))
+    W = rng.standard_normal((C, K))
+    A = rng.standard_normal((R, K))
+    B = rng.standard_normal((C, R))
+    z = rng.standard_normal(F * C * T)
+    s0, s1 = flow.SCHEDULE[1], flow.SCHEDULE[2]
+    got = flow.projection_euler_step(x, W, A, B, z, T, s0, s1)
+    for f in range(F):
+        for c in range(C):
+            for p in range(T):
+                m = f * T + p
+                v = sum(x[m, k] * W[c, k] for k in range(K))
+                v += sum(sum(x[m, k] * A[r, k] for k in range(K)) * B[c, r] for r in range(R))
+                i = (f * C + c) * T + p
+                assert abs(got[i] - (z[i] + (s1 - s0) * v)) <= 1e-12 * (1 + abs(z[i]) + abs(v))
+
+
+def test_projection_euler_recovers_z0():
+    """With x = I (one token per row of W) and W holding eps - z0 in token
+    order, three fused steps from the re-noised latent land on z0 -- the
+    closed form of the flow path -- only if tokens map to the right cells."""
+    rng = np.random.default_rng(32)
+    F, C, T = 3, 4, 6
+    M = F * T
+    z0 = rng.standard_normal((F, C, T))
+    eps = rng.standard_normal((F, C, T))
+    vel = (eps - z0).transpose(0, 2, 1).reshape(M, C)  # token-major velocity
+    x = np.eye(M)
+    W = vel.T
+    z = flow.renoise(z0, eps, flow.SCHEDULE[0])
+    for k in range(3):
+        z = flow.projection_euler_step(x, W, np.zeros((0, M)), np.zeros((C, 0)), z, T, flow.SCHEDULE[k],
+                                       flow.SCHEDULE[k + 1])
+    assert np.allclose(z, z0, rtol=0, atol=1e-14)
+    # The token-major layout read as channel-major misses.
+    wrong = flow.euler_step(flow.renoise(z0, eps, flow.SCHEDULE[0]), vel.reshape(F, C, T), flow.SCHEDULE[0], 0.0)
+    assert not np.allclose(wrong, z0, atol=1e-3)
+
+
+def test_projection_euler_zero_step_keeps_z():
+    rng = np.random.default_rng(33)
+    x = rng.standard_normal((8, 16))
+    W = rng.standard_normal((2, 16))
+    z = rng.standard_normal((2, 2, 4))
+    assert np.array_equal(flow.projection_euler_step(x, W, np.zeros((0, 16)), np.zeros((2, 0)), z, 4, 0.5, 0.5), z)
