@@ -299,6 +299,131 @@ def run_mxfp8(P, args, world, peaks):
     }
 
 
+def _time_calls(fn, reps, world):
+    """Mean ms of fn over reps calls (one untimed call first), CUDA events on
+    the current stream, max over ranks."""
+    fn()
+    torch.cuda.synchronize()
+    barrier(world)
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    t0.record()
+    for _ in range(reps):
+        fn()
+    t1.record()
+    torch.cuda.synchronize()
+    return max_over_ranks(t0.elapsed_time(t1) / reps, world)
+
+
+def run_fusions(P, args, world, peaks):
+    """Epilogue fusions beside the step, each against its unfused form:
+
+    * projection_euler: the step's last projection (d -> C channels, rank R)
+      with the Euler update and the bf16 copy of the new latent fused
+      (lg_lora_linear_euler), on all of the workload's whole frames; unfused:
+      lg_lora_linear with W padded to 32 rows, the velocity permuted into the
+      latent's layout by torch, lg_euler_step and a torch bf16 cast.
+    * swiglu_mxfp8: the MLP's input projection d -> 2 ffn with SwiGLU and the
+      MXFP8 quantizer fused (lg_lora_linear_swiglu_mxfp8) on a quarter of the
+      tokens (the unfused form holds the [M, 2 ffn] intermediate); unfused:
+      lg_lora_linear_mxfp8, torch silu(gate) * up in bf16, lg_mx_quantize.
+    """
+    import lora_gemm_b200 as lg
+    from lora_gemm_b200 import synth
+
+    w, dev, R = P.w, P.up.device, P.R
+    reps = max(args.steps, 2)
+    out = {}
+    L0 = P.layers[0]
+    K = L0["K"]
+    # Projection + Euler over whole frames of the layer-0 activations.
+    T = w.height * w.width
+    frames = P.M // T
+    if frames > 0 and K == w.d:
+        Kp, C = synth.proj_out_shape(w)
+        M = frames * T
+        x = L0["x"][:M]
+        W = synth.weight(w, synth.PROJ_OUT_LAYER, dev, shape=(Kp, C))
+        As, Bs = synth.adapters(w, synth.PROJ_OUT_LAYER, dev, shape=(Kp, C))
+        A_cat, B_cat = lg.lora_merge(As, Bs, P.scales)
+        z = torch.zeros((frames, C, T), dtype=torch.float32, device=dev)
+        zb = torch.empty_like(z, dtype=torch.bfloat16)
+        ws = torch.empty(lg.lora_linear_euler_workspace_size(M, K, C, R), dtype=torch.uint8, device=dev)
+        s0, s1 = P.sigmas[1], P.sigmas[2]
+        fused_ms = _time_calls(lambda: lg.lora_linear_euler(x, W, A_cat, B_cat, z, s0, s1, T, z_bf16=zb,
+                                                            workspace=ws), reps, world)
+        Cp = 32
+        Wp = torch.zeros((Cp, K), dtype=torch.bfloat16, device=dev)
+        Wp[:C] = W
+        Bp = torch.zeros((Cp, R), dtype=torch.float32, device=dev)
+        Bp[:C] = B_cat
+        y = torch.empty((M, Cp), dtype=torch.bfloat16, device=dev)
+        wsp = torch.empty(lg.lora_linear_workspace_size(M, K, Cp, R), dtype=torch.uint8, device=dev)
+
+        def unfused():
+            lg.lora_linear(x, Wp, A_cat, Bp, y=y, workspace=wsp)
+            v = y.view(frames, T, Cp)[:, :, :C].permute(0, 2, 1).float().contiguous()
+            lg.euler_step(z, v, s0, s1)
+            zb.copy_(z)
+
+        unfused_ms = _time_calls(unfused, reps, world)
+        fl = layer_flops(M, K, C, R)
+        peak = peaks["bf16_tflops_sustained"]
+        out["projection_euler"] = {
+            "workload": f"{w.name} last projection: {M} tokens ({frames} frames x {T} cells), d = {K} -> "
+                        f"{C} channels, rank {R}, FP32 latent + bf16 copy",
+            "fused_ms": round(fused_ms, 4), "unfused_ms": round(unfused_ms, 4),
+            "speedup": round(unfused_ms / fused_ms, 3),
+            "tflops": round(fl / (fused_ms * 1e-3) / 1e12, 1), "peak": peak,
+            "frac": round(fl / (fused_ms * 1e-3) / 1e12 / peak, 4),
+            "peak_kind": f"bf16_tflops_sustained ({peaks['source']}); algorithmic FLOPs with N = {C}",
+        }
+        del W, As, Bs, A_cat, B_cat, z, zb, ws, Wp, Bp, y, wsp
+    # SwiGLU + MXFP8 on a quarter of the tokens.
+    Km, N2 = synth.mlp_in_shape(w)
+    Mq = (P.M // 4) // 128 * 128 if P.M >= 512 else P.M
+    if K == Km and Mq > 0:
+        F = N2 // 2
+        x = L0["x"][:Mq]
+        W2 = synth.weight(w, synth.MLP_IN_LAYER, dev, shape=(Km, N2))
+        wq = lg.mx_quantize(W2)
+        del W2
+        As, Bs = synth.adapters(w, synth.MLP_IN_LAYER, dev, shape=(Km, N2))
+        A_cat, B_cat = lg.lora_merge(As, Bs, P.scales)
+        del As, Bs
+        xq = lg.mx_quantize(x)
+        q = (torch.empty((Mq, F), dtype=torch.uint8, device=dev),
+             torch.empty(lg.mx_scale_bytes(Mq, F), dtype=torch.uint8, device=dev))
+        ws = torch.empty(lg.lora_linear_workspace_size(Mq, Km, N2, R), dtype=torch.uint8, device=dev)
+        fused_ms = _time_calls(lambda: lg.lora_linear_swiglu_mxfp8(x, xq, wq, A_cat, B_cat, out=q, workspace=ws),
+                               reps, world)
+        y = torch.empty((Mq, N2), dtype=torch.bfloat16, device=dev)
+
+        def unfused():
+            lg.lora_linear_mxfp8(x, xq, wq, A_cat, B_cat, y=y, workspace=ws)
+            s = torch.nn.functional.silu(y[:, :F]) * y[:, F:]
+            lg.mx_quantize(s, codes=q[0], scales=q[1])
+
+        unfused_ms = _time_calls(unfused, reps, world)
+        fl = layer_flops(Mq, Km, N2, R)
+        peak = 2.0 * peaks["bf16_tflops_sustained"]
+        out["swiglu_mxfp8"] = {
+            "workload": f"{w.name} MLP input projection: {Mq} tokens (a quarter of the grid), d = {Km} -> 2 x {F} "
+                        f"(gate, up), rank {R}, MXFP8 output",
+            "fused_ms": round(fused_ms, 4), "unfused_ms": round(unfused_ms, 4),
+            "speedup": round(unfused_ms / fused_ms, 3),
+            "tflops": round(fl / (fused_ms * 1e-3) / 1e12, 1), "peak": round(peak, 1),
+            "frac": round(fl / (fused_ms * 1e-3) / 1e12 / peak, 4),
+            "peak_kind": "fp8 dense, derived: measured bf16 sustained x 2 (the nominal fp8 / bf16 ratio)",
+        }
+        del wq, A_cat, B_cat, xq, q, ws, y
+    torch.cuda.empty_cache()
+    status = lg.get_last_device_error()
+    if status != lg.LG_OK:
+        raise SystemExit(f"device error during the fusion runs: {lg.status_string(status)}")
+    return out
+
+
 def bytes_per_kernel(P):
     w = P.w
     n = w.latent_numel
@@ -434,6 +559,8 @@ def run_ours(args, rank, world, local):
     }
     if not args.no_mxfp8:
         result["mxfp8"] = run_mxfp8(P, args, world, peaks)
+    if not args.no_fusions:
+        result["fusions"] = run_fusions(P, args, world, peaks)
     if not args.no_e2e:
         result["e2e"] = run_e2e(P, args, world)
     if rank == 0 and not args.no_cpu_baseline:
@@ -712,6 +839,7 @@ def main():
     ap.add_argument("--workload", default=WORKLOAD)
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-mxfp8", action="store_true")
+    ap.add_argument("--no-fusions", action="store_true", help="skip the fused-epilogue comparisons")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--tokens", type=int, default=None,

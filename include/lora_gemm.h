@@ -212,6 +212,41 @@ lg_status lg_lora_linear_swiglu_mxfp8(const void* x, const void* x_codes, const 
                                       size_t ws_bytes, void* stream);
 
 /* ------------------------------------------------------------------------
+ * lg_lora_linear_euler -- the step's last projection (token activations to
+ * the latent's velocity channels) with the Euler update of "Open-H3-
+ * Regenerate-2K: High-Resolution Video Refinement with Few-Step Diffusion",
+ * section "Three steps instead of dozens", folded into its epilogue:
+ *
+ *   v = x W^T + (x A_cat^T) B_cat^T                    [M, N], FP32, not stored
+ *   z[f][c][p] = fmaf(sigma_next - sigma, v[f T + p][c], z[f][c][p])
+ *   z_bf16[f][c][p] = bf16(z[f][c][p])  (round to nearest even; next input)
+ *
+ * Token m is cell p = m mod T of frame f = m / T (T = frame_tokens, the H W
+ * cells of one latent frame), and the latent keeps its [frames, channels,
+ * cells] layout (the [F, C, H, W] latent with N = C channels).  The step
+ * sigma_next - sigma is rounded to FP32 first, as in lg_euler_step; v is the
+ * FP32 accumulator itself (lg_lora_linear would round it to bf16).
+ *
+ *   x, W, A_cat, B_cat  as for lg_lora_linear (W [N, K], B_cat [N, R]).
+ *   z       DEVICE [M / T, N, T] FP32, updated in place.
+ *   z_bf16  DEVICE [M / T, N, T] bf16, written; or NULL to skip the copy.
+ *   frame_tokens  T >= 1, M a multiple of T.
+ *   workspace, ws_bytes  at least lg_lora_linear_euler_workspace_size(M, K,
+ *          N, R) bytes (R = 0: none).
+ *
+ * Shapes: K and R as for lg_lora_linear; any N >= 1 (one tile covers
+ * N <= 224, and its MMAs then run with N rounded up to 16).  Variant as for
+ * lg_lora_linear (lg_set_kernel_variant applies: single-SM for K <= 2048,
+ * SM pairs beyond), always with one CTA or pair per panel
+ * (lg_set_cluster_size does not apply).  z and z_bf16 must not overlap each
+ * other, an input or the workspace.
+ * ---------------------------------------------------------------------- */
+size_t lg_lora_linear_euler_workspace_size(int64_t M, int K, int N, int R);
+lg_status lg_lora_linear_euler(const void* x, const void* W, const float* A_cat, const float* B_cat, float* z,
+                               void* z_bf16, int64_t M, int K, int N, int R, int64_t frame_tokens, float sigma,
+                               float sigma_next, void* workspace, size_t ws_bytes, void* stream);
+
+/* ------------------------------------------------------------------------
  * lg_lora_linear_noalloc -- lg_lora_linear for callers that cannot allocate
  * device memory.  The pages have no counterpart; this is an interface
  * addition of this library.

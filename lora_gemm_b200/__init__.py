@@ -57,6 +57,15 @@ _SIGNATURES = {
         [_c_void_p, _c_void_p, _c_void_p, _c_void_p, _c_void_p, _c_void_p, _c_void_p, _c_void_p, _c_void_p,
          ctypes.c_int64, ctypes.c_int, ctypes.c_int, ctypes.c_int, _c_void_p, ctypes.c_size_t, _c_void_p],
     ),
+    "lg_lora_linear_euler_workspace_size": (
+        ctypes.c_size_t, [ctypes.c_int64, ctypes.c_int, ctypes.c_int, ctypes.c_int]
+    ),
+    "lg_lora_linear_euler": (
+        ctypes.c_int,
+        [_c_void_p, _c_void_p, _c_void_p, _c_void_p, _c_void_p, _c_void_p, ctypes.c_int64, ctypes.c_int,
+         ctypes.c_int, ctypes.c_int, ctypes.c_int64, ctypes.c_float, ctypes.c_float, _c_void_p, ctypes.c_size_t,
+         _c_void_p],
+    ),
     "lg_lora_linear_noalloc": (
         ctypes.c_int,
         [_c_void_p, _c_void_p, _c_void_p, _c_void_p, _c_void_p, ctypes.c_int64, ctypes.c_int, ctypes.c_int,
@@ -324,6 +333,50 @@ def lora_linear_swiglu_mxfp8(x, x_mx, W2_mx, A_cat, B_cat, out=None, workspace=N
                                              ws_bytes, _stream(x.device))
     _check(st, "lg_lora_linear_swiglu_mxfp8")
     return out
+
+
+def lora_linear_euler_workspace_size(M, K, N, R):
+    return int(lib.lg_lora_linear_euler_workspace_size(int(M), int(K), int(N), int(R)))
+
+
+def lora_linear_euler(x, W, A_cat, B_cat, z, sigma, sigma_next, frame_tokens, z_bf16=None, workspace=None):
+    """The step's last projection with the Euler update fused: v = x W^T +
+    (x A_cat^T) B_cat^T (W [C, K]) updates the FP32 latent z [frames, C,
+    frame_tokens] in place, z += (sigma_next - sigma) v (token m = cell
+    m mod frame_tokens of frame m // frame_tokens); z_bf16 (same shape, or
+    None) receives bf16(z).  Returns z."""
+    _need(x, torch.bfloat16, "x", 2)
+    _need(W, torch.bfloat16, "W", 2)
+    _need(z, torch.float32, "z")
+    M, K = x.shape
+    N = W.shape[0]
+    if W.shape[1] != K:
+        raise ValueError("W must be [N, K]")
+    if z.numel() != M * N:
+        raise ValueError("z must hold M * N elements")
+    if z_bf16 is not None:
+        _need(z_bf16, torch.bfloat16, "z_bf16")
+        if z_bf16.numel() != z.numel():
+            raise ValueError("z_bf16 must have as many elements as z")
+    R = 0
+    if A_cat is not None and A_cat.numel() > 0:
+        _need(A_cat, torch.float32, "A_cat", 2)
+        _need(B_cat, torch.float32, "B_cat", 2)
+        R = A_cat.shape[0]
+        if A_cat.shape[1] != K or tuple(B_cat.shape) != (N, R):
+            raise ValueError("A_cat must be [R, K] and B_cat [N, R]")
+    else:
+        A_cat = B_cat = None
+    need = lora_linear_euler_workspace_size(M, K, N, R)
+    if workspace is None and need > 0:
+        workspace = torch.empty(need, dtype=torch.uint8, device=x.device)
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    with torch.cuda.device(x.device):
+        st = lib.lg_lora_linear_euler(_ptr(x), _ptr(W), _ptr(A_cat), _ptr(B_cat), _ptr(z), _ptr(z_bf16), M, K, N, R,
+                                      int(frame_tokens), float(sigma), float(sigma_next), _ptr(workspace), ws_bytes,
+                                      _stream(x.device))
+    _check(st, "lg_lora_linear_euler")
+    return z
 
 
 def lora_linear_noalloc(x, W, A_cat, B_cat, y):

@@ -180,11 +180,23 @@ lg_status lg_mx_quantize(const void* in, int64_t rows, int K, void* codes, void*
                   1);
 }
 
+namespace {
+// bf16 copies of A_cat [R, K] and B_cat [N, R], each padded to 256 bytes.
+size_t factor_copy_bytes(int K, int N, int R) { return (size_t)(align256(2ull * R * K) + align256(2ull * N * R)); }
+}  // namespace
+
 size_t lg_lora_linear_workspace_size(int64_t M, int K, int N, int R) {
   if (M < 0 || K < 64 || N < 32 || K % 64 || N % 32 || K > kMaxDim || N > kMaxDim) return 0;
   if (R < 0 || R % 64 || R > kMaxRank) return 0;
   if (R == 0) return 0;
-  return (size_t)(align256(2ull * R * K) + align256(2ull * N * R));
+  return factor_copy_bytes(K, N, R);
+}
+
+size_t lg_lora_linear_euler_workspace_size(int64_t M, int K, int N, int R) {
+  if (M < 0 || K < 64 || N < 1 || K % 64 || K > kMaxDim || N > kMaxDim) return 0;
+  if (R < 0 || R % 64 || R > kMaxRank) return 0;
+  if (R == 0) return 0;
+  return factor_copy_bytes(K, N, R);
 }
 
 namespace {
@@ -203,11 +215,21 @@ struct SwigluOut {
   void* scales;
 };
 
+// Fused Euler output of lg_lora_linear_euler (null otherwise).
+struct EulerOut {
+  float* z;
+  void* z_bf16;
+  int64_t frame_tokens;
+  float dt;
+};
+
 lg_status lora_linear_impl(const void* x, const void* W, const float* A_cat, const float* B_cat, void* y, int64_t M,
                            int K, int N, int R, void* workspace, size_t ws_bytes, void* stream,
-                           const MxOperands* mx, const SwigluOut* sw = nullptr) {
+                           const MxOperands* mx, const SwigluOut* sw = nullptr, const EulerOut* eu = nullptr) {
   if (M < 0 || K < 0 || N < 0 || R < 0) return LG_ERR_INVALID_ARG;
-  if (M >= (int64_t)1 << 31 || K < 64 || N < 32 || K % 64 || N % 32 || K > kMaxDim || N > kMaxDim)
+  // The Euler output takes any N >= 1 (its epilogue writes single values).
+  const bool n_ok = eu ? N >= 1 : (N >= 32 && N % 32 == 0);
+  if (M >= (int64_t)1 << 31 || K < 64 || !n_ok || K % 64 || K > kMaxDim || N > kMaxDim)
     return LG_ERR_UNSUPPORTED_SHAPE;
   if (R % 64 || R > kMaxRank) return LG_ERR_UNSUPPORTED_SHAPE;
   if (mx && K % 128) return LG_ERR_UNSUPPORTED_SHAPE;
@@ -216,22 +238,35 @@ lg_status lora_linear_impl(const void* x, const void* W, const float* A_cat, con
     if (!sw->codes || !sw->scales) return LG_ERR_INVALID_ARG;
     if (!aligned16(sw->codes) || !aligned16(sw->scales)) return LG_ERR_MISALIGNED;
   }
-  if (!x || (!sw && !y) || (!mx && !W)) return LG_ERR_INVALID_ARG;
+  if (eu) {
+    if (!eu->z || eu->frame_tokens < 1 || M % eu->frame_tokens || !std::isfinite(eu->dt)) return LG_ERR_INVALID_ARG;
+    if (!aligned16(eu->z) || (eu->z_bf16 && !aligned16(eu->z_bf16))) return LG_ERR_MISALIGNED;
+  }
+  const bool no_y = sw || eu;
+  if (!x || (!no_y && !y) || (!mx && !W)) return LG_ERR_INVALID_ARG;
   if (mx && (!mx->xq || !mx->xsf || !mx->wq || !mx->wsf)) return LG_ERR_INVALID_ARG;
   if (R > 0 && (!A_cat || !B_cat)) return LG_ERR_INVALID_ARG;
-  if (!aligned16(x) || (!sw && !aligned16(y)) || (!mx && !aligned16(W))) return LG_ERR_MISALIGNED;
+  if (!aligned16(x) || (!no_y && !aligned16(y)) || (!mx && !aligned16(W))) return LG_ERR_MISALIGNED;
   if (mx && (!aligned16(mx->xq) || !aligned16(mx->xsf) || !aligned16(mx->wq) || !aligned16(mx->wsf)))
     return LG_ERR_MISALIGNED;
   if (R > 0 && (!aligned16(A_cat) || !aligned16(B_cat))) return LG_ERR_MISALIGNED;
-  const size_t need = lg_lora_linear_workspace_size(M, K, N, R);
+  const size_t need = R > 0 ? factor_copy_bytes(K, N, R) : 0;
   if (R > 0) {
     if (!workspace || ws_bytes < need) return LG_ERR_WORKSPACE;
     if (!aligned16(workspace)) return LG_ERR_MISALIGNED;
   }
   const uint64_t bx = 2ull * M * K, bw = 2ull * N * K;
-  // The output region: y, or the SwiGLU codes and scales.
-  const void* out = sw ? sw->codes : y;
-  const uint64_t by = sw ? 1ull * M * (N / 2) : 2ull * M * N;
+  // The output region: y, the SwiGLU codes and scales, or the latent z (and
+  // its bf16 copy, checked here).
+  const void* out = sw ? sw->codes : (eu ? eu->z : y);
+  const uint64_t by = sw ? 1ull * M * (N / 2) : (eu ? 4ull * M * N : 2ull * M * N);
+  if (eu && eu->z_bf16 && M > 0) {
+    const uint64_t bb = 2ull * M * N;
+    if (overlaps(eu->z_bf16, bb, eu->z, by) || overlaps(eu->z_bf16, bb, x, bx) || overlaps(eu->z_bf16, bb, W, bw) ||
+        (R > 0 && (overlaps(eu->z_bf16, bb, A_cat, 4ull * R * K) || overlaps(eu->z_bf16, bb, B_cat, 4ull * N * R) ||
+                   overlaps(eu->z_bf16, bb, workspace, need))))
+      return LG_ERR_INVALID_ARG;
+  }
   if (sw && M > 0) {
     const uint64_t bs = lg_mx_scale_bytes(M, N / 2);
     if (overlaps(sw->codes, by, sw->scales, bs) || overlaps(sw->scales, bs, x, bx) ||
@@ -284,6 +319,13 @@ lg_status lora_linear_impl(const void* x, const void* W, const float* A_cat, con
     p.wq = mx->wq;
     p.wsf = mx->wsf;
   }
+  if (eu) {
+    p.y = nullptr;
+    p.eu_z = eu->z;
+    p.eu_zb = eu->z_bf16;
+    p.eu_frame = eu->frame_tokens;
+    p.eu_dt = eu->dt;
+  }
   if (sw) {
     p.y = nullptr;
     p.ffn = N / 2;
@@ -319,6 +361,15 @@ lg_status lg_lora_linear_swiglu_mxfp8(const void* x, const void* x_codes, const 
   const MxOperands mx{x_codes, x_scales, W_codes, W_scales};
   const SwigluOut sw{out_codes, out_scales};
   return lora_linear_impl(x, nullptr, A_cat, B_cat, nullptr, M, K, 2 * F, R, workspace, ws_bytes, stream, &mx, &sw);
+}
+
+lg_status lg_lora_linear_euler(const void* x, const void* W, const float* A_cat, const float* B_cat, float* z,
+                               void* z_bf16, int64_t M, int K, int N, int R, int64_t frame_tokens, float sigma,
+                               float sigma_next, void* workspace, size_t ws_bytes, void* stream) {
+  if (!std::isfinite(sigma) || !std::isfinite(sigma_next)) return LG_ERR_INVALID_ARG;
+  // The step is taken in FP32, as lg_euler_step takes it.
+  const EulerOut eu{z, z_bf16, frame_tokens, sigma_next - sigma};
+  return lora_linear_impl(x, W, A_cat, B_cat, nullptr, M, K, N, R, workspace, ws_bytes, stream, nullptr, nullptr, &eu);
 }
 
 lg_status lg_renoise(const float* up, float* x, int64_t n, float sigma, uint64_t seed, uint64_t offset,

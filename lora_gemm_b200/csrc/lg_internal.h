@@ -70,6 +70,12 @@ struct LinearLaunch {
   int ffn = 0;
   void* q_codes = nullptr;
   void* q_scales = nullptr;
+  // Fused Euler update (bf16 layer only): y is not
+  // written; z [M / eu_frame, N, eu_frame] += eu_dt v, bf16 copy to eu_zb.
+  float* eu_z = nullptr;
+  void* eu_zb = nullptr;
+  int64_t eu_frame = 0;
+  float eu_dt = 0.f;
 };
 // Returns cudaSuccess or the failing CUDA error; *driver_failed is set when
 // the tensor-map encoder (driver API) is missing or rejects a map.

@@ -164,6 +164,17 @@ struct Args {
   int ffn;
   uint8_t* q_codes;   // [M, ffn]
   uint8_t* q_scales;  // blocked layout, ffn / 128 K groups
+  // MMA N of the output tiles: BN, or N rounded up to 16 when one tile
+  // covers all N columns (the rest of the tile would be zeros); bf16 only.
+  int y_n;
+  // Euler output (bf16 variants, eu_z != null): v = the FP32 accumulator
+  // is not stored; token m's channel c updates the latent z [M / eu_frame, N,
+  // eu_frame] in place, z += eu_dt v, and eu_zb (if not null) receives the
+  // bf16 copy of the updated z in the same layout.
+  float* eu_z;
+  uint16_t* eu_zb;
+  int64_t eu_frame;
+  float eu_dt;
   unsigned long long wait_limit_ns;
 };
 
@@ -302,7 +313,8 @@ __device__ void run_producer(const CUtensorMap* tm_x, const CUtensorMap* tm_w, c
       fence_proxy_async_smem();
     }
     for (int t = member; ok && t < a.n_tiles; t += a.group, ++sweep) {
-      const int n0 = a.ffn > 0 ? (half ? a.ffn : 0) + t * BM : t * C::BN + half * (int)C::B_ROWS;
+      // A pair's MMA takes y_n / 2 B rows from each CTA (B_ROWS when y_n = BN).
+      const int n0 = a.ffn > 0 ? (half ? a.ffn : 0) + t * BM : t * C::BN + half * (a.y_n / 2);
       const int kloop = MX ? a.kq_blocks : a.k_blocks;
       for (int i = 0; i < kloop; ++i) {
         const int kb = (sweep & 1) ? kloop - 1 - i : i;
@@ -376,7 +388,7 @@ __device__ void run_mma(const Args& a, Control* ctl, uint32_t smem_base, uint32_
   const uint32_t acc_full = smem_u32(&ctl->acc_full);
   const uint32_t acc_empty = smem_u32(&ctl->acc_empty);
   const uint32_t idesc_h = idesc_bf16_f32(C::MMA_M, a.chunk_n);
-  constexpr uint32_t idesc_y = idesc_bf16_f32(C::MMA_M, C::BN);
+  const uint32_t idesc_y = idesc_bf16_f32(C::MMA_M, a.y_n);
   const uint32_t d_acc = tmem + ACC_COL;
   auto commit = [&](uint32_t bar) {
     if constexpr (PAIR) {
@@ -662,6 +674,41 @@ __device__ __forceinline__ void swiglu_quantize_store(const Args& a, int64_t row
   }
 }
 
+// Euler update for one token row: z[f][col][p] = fmaf(dt, v[col], z[f][col][p])
+// for the `cols` accumulator columns col0 .. col0 + cols - 1 below N, with f
+// and p the row's frame and cell; the bf16 (round to nearest even) copy of
+// the new value goes to eu_zb.  The 32 lanes of a warp hold 32 consecutive
+// tokens, so each column is one coalesced 128-byte access per warp (two at a
+// frame boundary).  Per 16 columns all loads are issued before any store.
+template <int CHUNKS>
+__device__ __forceinline__ void euler_store(const Args& a, int64_t row, int col0, int cols,
+                                            const uint32_t (&v)[CHUNKS][16]) {
+  if (row >= a.M) return;
+  const int64_t f = row / a.eu_frame;
+  float* z = a.eu_z + f * a.N * a.eu_frame + (row - f * a.eu_frame);
+  uint16_t* zb = a.eu_zb ? a.eu_zb + (z - a.eu_z) : nullptr;
+#pragma unroll
+  for (int i = 0; i < CHUNKS; ++i) {
+    if (16 * i >= cols) break;
+    float old[16];
+#pragma unroll
+    for (int j = 0; j < 16; ++j) {
+      const int c = 16 * i + j;
+      old[j] = (c < cols && col0 + c < a.N) ? z[(int64_t)(col0 + c) * a.eu_frame] : 0.f;
+    }
+#pragma unroll
+    for (int j = 0; j < 16; ++j) {
+      const int c = 16 * i + j;
+      if (c < cols && col0 + c < a.N) {
+        const int64_t off = (int64_t)(col0 + c) * a.eu_frame;
+        const float zn = fmaf(a.eu_dt, __uint_as_float(v[i][j]), old[j]);
+        z[off] = zn;
+        if (zb) zb[off] = __bfloat16_as_ushort(__float2bfloat16_rn(zn));
+      }
+    }
+  }
+}
+
 // ---------------------------------------------------------------------------
 // Epilogue (warps 2..9): warp w reads TMEM lanes 32 (w mod 4) .. +31 and
 // handles half (w - 2) / 4 of the columns.
@@ -773,6 +820,36 @@ __device__ void run_epilogue(const CUtensorMap* tm_y, const Args& a, Control* ct
           tmem_wait_ld();
           release_acc(false);
           swiglu_quantize_store(a, m0 + row_in_tile, t * BM + 64 * half, g, u);
+          continue;
+        }
+      }
+      if constexpr (!MX) {
+        if (a.eu_z) {
+          // Euler output: this warp's y_n / 2 columns (a multiple of 8; a
+          // 16-column load past them reads accumulator columns it ignores).
+          // Up to 32 columns (N <= 64) go to registers and the accumulator is
+          // handed back before the stores; wider tiles are stored 16 columns
+          // at a time and hand it back at the end.
+          const int cols = a.y_n / 2;
+          const uint32_t src = lane_base + ACC_COL + (uint32_t)(half * cols);
+          const int col0 = t * C::BN + half * cols;
+          const int64_t row = m0 + row_in_tile;
+          if (cols <= 32) {
+            uint32_t v[2][16];
+            tmem_ld_32x32b_x16(src, v[0]);
+            if (cols > 16) tmem_ld_32x32b_x16(src + 16, v[1]);
+            tmem_wait_ld();
+            release_acc(false);
+            euler_store<2>(a, row, col0, cols, v);
+          } else {
+            for (int c = 0; c < cols; c += 16) {
+              uint32_t v[1][16];
+              tmem_ld_32x32b_x16(src + (uint32_t)c, v[0]);
+              tmem_wait_ld();
+              euler_store<1>(a, row, col0 + c, min(16, cols - c), v);
+            }
+            release_acc(false);
+          }
           continue;
         }
       }
@@ -1124,10 +1201,12 @@ cudaError_t launch_variant(const LinearLaunch& p, cudaStream_t s, int dev, int c
     tm_sfb = tm_x;
   }
   if (ok) {
-    if (PAIR && p.ffn == 0) {
+    if (PAIR && p.ffn == 0 && !p.eu_z) {
       ok = make_store_map(enc, &tm_y, p.y, (uint64_t)p.N, (uint64_t)p.M);
     } else {
-      tm_y = tm_x;  // never used: the single-SM epilogue stores directly, SwiGLU writes MXFP8
+      // Never used: the single-SM epilogue stores directly, SwiGLU writes
+      // MXFP8, the Euler output updates the latent.
+      tm_y = tm_x;
     }
   }
   if (ok && p.R > 0) {
@@ -1149,6 +1228,11 @@ cudaError_t launch_variant(const LinearLaunch& p, cudaStream_t s, int dev, int c
   args.num_panels = (int)((p.M + C::PANEL - 1) / C::PANEL);
   args.n_tiles = p.ffn > 0 ? p.ffn / BM : (p.N + C::BN - 1) / C::BN;
   args.ffn = p.ffn;
+  args.y_n = (!MX && args.n_tiles == 1) ? (p.N + 15) / 16 * 16 : C::BN;
+  args.eu_z = p.eu_z;
+  args.eu_zb = reinterpret_cast<uint16_t*>(p.eu_zb);
+  args.eu_frame = p.eu_frame;
+  args.eu_dt = p.eu_dt;
   args.q_codes = reinterpret_cast<uint8_t*>(p.q_codes);
   args.q_scales = reinterpret_cast<uint8_t*>(p.q_scales);
   args.k_blocks = p.K / BK;
@@ -1219,8 +1303,17 @@ cudaError_t launch_lora_linear(const LinearLaunch& p, cudaStream_t s, bool* driv
       if (cluster == 0) cluster = 1;
     } else {
       variant = 2;
-      if (cluster == 0) cluster = p.K <= 4096 ? 2 : 4;
+      // Two pairs per panel only when there are N tiles for both.
+      if (cluster == 0) cluster = (p.K <= 4096 || p.N <= 256) ? 2 : 4;
     }
+  }
+  if (p.eu_z) {
+    // The Euler output keeps one CTA (or one pair) per panel: its tiles are
+    // few (one for N <= 224), so members sharing a panel would idle.  Pairs
+    // for K > 2048 as above (each CTA loads half of every A_cat chunk).
+    const int v = g_variant_override.load(std::memory_order_relaxed);
+    if (v == 1 || (v == 0 && p.K <= 2048)) return launch_variant<false, false>(p, s, dev, 1, driver_failed, enc);
+    return launch_variant<true, false>(p, s, dev, 2, driver_failed, enc);
   }
   if (p.mx) {
     // The MXFP8 base term runs on SM pairs only.

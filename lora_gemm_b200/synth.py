@@ -121,16 +121,17 @@ def activations(w, K, layer, device, M=None):
     return fill_normal_(x, 1.0, generator(w.seed, _STREAM_X + layer, device))
 
 
-def weight(w, layer, device):
-    """W ~ N(0, 1/K), bf16 [N, K]."""
-    K, N = w.shapes[layer]
+def weight(w, layer, device, shape=None):
+    """W ~ N(0, 1/K), bf16 [N, K]; shape = (K, N) overrides the layer's."""
+    K, N = w.shapes[layer] if shape is None else shape
     W = torch.empty((N, K), dtype=torch.bfloat16, device=device)
     return fill_normal_(W, K ** -0.5, generator(w.seed, _STREAM_W + layer, device))
 
 
-def adapters(w, layer, device, ranks=ADAPTER_RANKS):
-    """A_i ~ N(0, 1/K) [r_i, K] and B_i ~ N(0, 0.01) [N, r_i], FP32."""
-    K, N = w.shapes[layer]
+def adapters(w, layer, device, ranks=ADAPTER_RANKS, shape=None):
+    """A_i ~ N(0, 1/K) [r_i, K] and B_i ~ N(0, 0.01) [N, r_i], FP32; shape =
+    (K, N) overrides the layer's."""
+    K, N = w.shapes[layer] if shape is None else shape
     As, Bs = [], []
     for i, r in enumerate(ranks):
         A = torch.empty((r, K), dtype=torch.float32, device=device)
@@ -140,6 +141,23 @@ def adapters(w, layer, device, ranks=ADAPTER_RANKS):
         As.append(A)
         Bs.append(B)
     return As, Bs
+
+
+# Extra projections around the three layers, drawn on their own streams
+# (layer index past the workload's shapes):
+#   the step's last projection, d -> C velocity channels per token;
+#   the MLP's input projection with SwiGLU, d -> 2 ffn (gate rows, then up
+#   rows), ffn = 4 d (the 4d -> d layer's input width).
+PROJ_OUT_LAYER = 10
+MLP_IN_LAYER = 11
+
+
+def proj_out_shape(w):
+    return (w.d, w.channels)
+
+
+def mlp_in_shape(w):
+    return (w.d, 8 * w.d)
 
 
 def upscaled_latent(w, device):

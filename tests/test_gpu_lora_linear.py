@@ -207,3 +207,19 @@ def test_cluster_size_argument_checked():
         lg.set_cluster_size(16)
     with pytest.raises(lg.LoraGemmError):
         lg.set_kernel_variant(3)
+
+
+@pytest.mark.parametrize("variant", [1, 2])
+@pytest.mark.parametrize("N", [32, 96, 160, 224])
+def test_narrow_n_single_tile(variant, N):
+    """N below the tile width: one output tile whose MMAs run with N columns
+    (an SM pair takes N / 2 B rows from each CTA)."""
+    x, W, A, B = _rand_layer(700, 512, N, 576, seed=N + variant)
+    lg.set_kernel_variant(variant)
+    try:
+        y = lg.lora_linear(x, W, A, B)
+        err = _check(x, W, A, B, y)
+    finally:
+        lg.set_kernel_variant(0)
+    assert lg.get_last_device_error() == lg.LG_OK
+    assert err <= TOL, err
