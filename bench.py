@@ -768,13 +768,23 @@ class OracleStep:
         return z
 
 
+def _oracle_tokens_for(w, seconds, cap):
+    """Tokens whose OracleStep takes about `seconds`: a fixed cost (the
+    merge, per-layer setup) plus a per-token cost, fitted from two probes."""
+    times = []
+    for n in (32, 256):
+        probe = OracleStep(w, n)
+        probe.run()
+        t0 = time.perf_counter()
+        probe.run()
+        times.append(time.perf_counter() - t0)
+    per_token = max((times[1] - times[0]) / 224.0, 1e-7)
+    fixed = max(times[0] - 32 * per_token, 0.0)
+    return int(max(32, min(cap, (seconds - fixed) / per_token)))
+
+
 def cpu_baseline(w, target_s=15.0):
-    probe = OracleStep(w, 32)
-    probe.run()
-    t0 = time.perf_counter()
-    probe.run()
-    t_probe = time.perf_counter() - t0
-    tokens = int(max(32, min(4096, 32 * target_s / max(t_probe, 1e-3))))
+    tokens = _oracle_tokens_for(w, target_s, 12288)
     step = OracleStep(w, tokens)
     t0 = time.perf_counter()
     step.run()
@@ -788,13 +798,8 @@ def run_reference(args, rank, world):
     from lora_gemm_b200 import synth
 
     w = synth.WORKLOADS[args.workload]
-    probe = OracleStep(w, 32)
-    probe.run()
-    t0 = time.perf_counter()
-    probe.run()
-    t_probe = time.perf_counter() - t0
     per_step_s = 90.0 / max(1, args.steps + args.warmup)
-    tokens = int(max(32, min(2048, 32 * per_step_s / max(t_probe, 1e-3))))
+    tokens = _oracle_tokens_for(w, per_step_s, 12288)
     step = OracleStep(w, tokens)
     for _ in range(args.warmup):
         step.run()
