@@ -282,6 +282,7 @@ def run_mxfp8(P, args, world, peaks):
     tflops = sum(flops) / (sum(lin_ms) * 1e-3) / 1e12
     fp8_peak = 2.0 * peaks["bf16_tflops_sustained"]
     q_ms = sum(per["quantize"]) / args.steps
+    cublas = _cublas_mxfp8_context(P, xq, wq, world)
     del xq, wq
     return {
         "value": round(_dist().whole_job_rate(P.M, world, args.steps, ms), 1), "unit": UNIT,
@@ -295,8 +296,31 @@ def run_mxfp8(P, args, world, peaks):
             "frac": round(tflops / fp8_peak, 4),
         },
         "quantize_x_ms_per_step": round(q_ms, 4),
+        "cublas_mxfp8_base_term": cublas,
         "note": "W quantized once outside the timed steps; x quantized inside; LoRA path bf16",
     }
+
+
+def _cublas_mxfp8_context(P, xq, wq, world):
+    """Context for the MXFP8 layers: cuBLAS's block-scaled MXFP8 GEMM
+    (torch._scaled_mm) on the same codes and scales -- the scale layout
+    lg_mx_quantize writes is the one cuBLAS takes -- computing the base term
+    deq(x) deq(W)^T alone, without the LoRA term, per layer shape."""
+    try:
+        layers = []
+        for k, L in enumerate(P.layers):
+            a, sa = xq[id(L["x"])]
+            b, sb = wq[k]
+            A8, B8 = a.view(torch.float8_e4m3fn), b.view(torch.float8_e4m3fn)
+            SA, SB = sa.view(torch.float8_e8m0fnu), sb.view(torch.float8_e8m0fnu)
+            ms = _time_calls(lambda: torch._scaled_mm(A8, B8.t(), scale_a=SA, scale_b=SB, out_dtype=torch.bfloat16),
+                             2, world)
+            layers.append({"ms": round(ms, 4), "tflops": round(2.0 * P.M * L["K"] * L["N"] / (ms * 1e-3) / 1e12, 1)})
+        torch.cuda.empty_cache()
+        return {"per_layer": layers, "what": "torch._scaled_mm, E4M3 codes with E8M0 block scales (1 x 32), "
+                                             "base term only (no LoRA), bf16 output"}
+    except Exception as e:  # an older torch or cuBLAS without MXFP8
+        return {"unavailable": f"{type(e).__name__}: {str(e)[:200]}"}
 
 
 def _time_calls(fn, reps, world):

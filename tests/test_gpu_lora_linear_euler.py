@@ -157,3 +157,25 @@ def test_rejects_bad_arguments():
     with pytest.raises(lg.LoraGemmError) as ei:
         lg.lora_linear_euler(x, W, A, B, z, S0, S1, 256, z_bf16=x.view(-1)[: z.numel()])   # copy over x
     assert ei.value.status == lg.LG_ERR_INVALID_ARG
+
+
+@pytest.mark.parametrize("variant", [1, 2])
+def test_wait_timeout_is_reported(variant):
+    """A 1 ns wait limit makes the pipeline's waits run out: the status says so
+    and the next call with the default limit is correct."""
+    x, W, A, B, z = _case(2, 1024, 24, 2048, 576, seed=23)
+    lg.set_kernel_variant(variant)
+    try:
+        lg.set_wait_limit_ns(1)
+        try:
+            lg.lora_linear_euler(x, W, A, B, z.clone(), S0, S1, 1024)
+            status = lg.get_last_device_error()
+        finally:
+            lg.set_wait_limit_ns(0)
+        z_old = z.clone()
+        lg.lora_linear_euler(x, W, A, B, z, S0, S1, 1024)
+    finally:
+        lg.set_kernel_variant(0)
+    assert status == lg.LG_ERR_DEVICE_TIMEOUT
+    assert lg.get_last_device_error() == lg.LG_OK
+    _check(x, W, A, B, 576, z_old, z, None, 1024)

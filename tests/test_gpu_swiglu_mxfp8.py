@@ -107,3 +107,19 @@ def test_swiglu_rejects_bad_ffn():
         lg.lora_linear_swiglu_mxfp8(x, (codes[:8], sc), (codes, sc), None, None,
                                     out=(torch.zeros(8, 96, dtype=torch.uint8, device=DEV), sc))
     assert ei.value.status == lg.LG_ERR_UNSUPPORTED_SHAPE
+
+
+def test_swiglu_wait_timeout_is_reported():
+    M, K, F, R = 2048, 1024, 512, 576
+    x, W2, A, B = _layer(M, K, F, R, seed=77)
+    xq, wq = lg.mx_quantize(x), lg.mx_quantize(W2)
+    lg.set_wait_limit_ns(1)
+    try:
+        lg.lora_linear_swiglu_mxfp8(x, xq, wq, A, B)
+        status = lg.get_last_device_error()
+    finally:
+        lg.set_wait_limit_ns(0)
+    assert status == lg.LG_ERR_DEVICE_TIMEOUT
+    codes, scales = lg.lora_linear_swiglu_mxfp8(x, xq, wq, A, B)
+    assert lg.get_last_device_error() == lg.LG_OK
+    _check(x, W2, A, B, R, codes, scales)
