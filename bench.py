@@ -339,6 +339,51 @@ def _time_calls(fn, reps, world):
     return max_over_ranks(t0.elapsed_time(t1) / reps, world)
 
 
+def run_ic_routes(P, args, world, peaks):
+    """The IC sampler routes (up3, up4, hf8: re-noise at the route's start and
+    one Euler step per rung of HyperFlow's shift-12 ladder) on the workload's
+    latent, with the step's velocity stand-ins.  The linear layers of each
+    rung are those of the main step and are not repeated here.  L2 is flushed
+    (a 256 MiB write) before every timed route; only the route is timed."""
+    import lora_gemm_b200 as lg
+
+    hbm = peaks["hbm_gbs"]
+    n = P.up.numel()
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=P.up.device)
+    out = {}
+    for route, s0 in lg.IC_ROUTES.items():
+        lad = lg.shift_ladder(s0)
+
+        def f(lad=lad):
+            lg.renoise(P.up, lad[0], P.w.seed, offset=P.noise_offset, out=P.x_lat)
+            for k in range(len(lad) - 1):
+                lg.euler_step(P.x_lat, P.v[k % len(P.v)], lad[k], lad[k + 1])
+
+        f()
+        times = []
+        for _ in range(max(args.steps, 5)):
+            flush.zero_()
+            e0 = torch.cuda.Event(enable_timing=True)
+            e1 = torch.cuda.Event(enable_timing=True)
+            e0.record()
+            f()
+            e1.record()
+            torch.cuda.synchronize()
+            times.append(e0.elapsed_time(e1))
+        ms = max_over_ranks(statistics.median(times), world)
+        nbytes = 8.0 * n + 12.0 * n * (len(lad) - 1)
+        out[route] = {"sigmas": [round(x, 6) for x in lad], "euler_steps": len(lad) - 1, "ms": round(ms, 4),
+                      "gbs": round(nbytes / (ms * 1e-3) / 1e9, 1),
+                      "frac_of_measured_hbm": round(nbytes / (ms * 1e-3) / 1e9 / hbm, 4)}
+    del flush
+    status = lg.get_last_device_error()
+    if status != lg.LG_OK:
+        raise SystemExit(f"device error during the IC routes: {lg.status_string(status)}")
+    out["note"] = (f"algorithmic bytes 8 + 12 per step per latent element; the {4 * n / 1e6:.0f} MB latent stays "
+                   "partly in L2 between the steps of a route, so long routes can pass the HBM copy rate")
+    return out
+
+
 def run_fusions(P, args, world, peaks):
     """Epilogue fusions beside the step, each against its unfused form:
 
@@ -585,6 +630,7 @@ def run_ours(args, rank, world, local):
         result["mxfp8"] = run_mxfp8(P, args, world, peaks)
     if not args.no_fusions:
         result["fusions"] = run_fusions(P, args, world, peaks)
+        result["ic_routes"] = run_ic_routes(P, args, world, peaks)
     if not args.no_e2e:
         result["e2e"] = run_e2e(P, args, world)
     if rank == 0 and not args.no_cpu_baseline:
@@ -808,7 +854,7 @@ def _oracle_tokens_for(w, seconds, cap):
 
 
 def cpu_baseline(w, target_s=15.0):
-    tokens = _oracle_tokens_for(w, target_s, 12288)
+    tokens = _oracle_tokens_for(w, target_s, 16384)
     step = OracleStep(w, tokens)
     t0 = time.perf_counter()
     step.run()
@@ -868,7 +914,7 @@ def main():
     ap.add_argument("--workload", default=WORKLOAD)
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-mxfp8", action="store_true")
-    ap.add_argument("--no-fusions", action="store_true", help="skip the fused-epilogue comparisons")
+    ap.add_argument("--no-fusions", action="store_true", help="skip the fused-epilogue comparisons and the IC routes")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--tokens", type=int, default=None,
