@@ -140,6 +140,32 @@ def _need(t, dtype, name, ndim=None):
         raise ValueError(f"{name} must have {ndim} dimensions")
 
 
+def _shape(t, shape, name):
+    if tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} must have shape {tuple(shape)}, got {tuple(t.shape)}")
+
+
+def _at_least(t, nbytes, name):
+    _need(t, torch.uint8, name)
+    if t.numel() < nbytes:
+        raise ValueError(f"{name} holds {t.numel()} bytes, needs {nbytes}")
+
+
+def _same_device(ref, *tensors):
+    """Every tensor given (None skipped) on ref's device: the kernels run there."""
+    for t in tensors:
+        if t is not None and t.device != ref.device:
+            raise ValueError(f"all tensors must be on {ref.device}, got one on {t.device}")
+
+
+def _scales(pair, rows, K, what):
+    codes, sc = pair
+    _need(codes, torch.uint8, f"{what} codes", 2)
+    _shape(codes, (rows, K), f"{what} codes")
+    _at_least(sc, mx_scale_bytes(rows, K), f"{what} scales")
+    return codes, sc
+
+
 def status_string(status):
     return lib.lg_status_string(int(status)).decode()
 
@@ -197,6 +223,9 @@ def lora_merge(As, Bs, scales, A_cat=None, B_cat=None):
         B_cat = torch.empty((d_out, R), dtype=torch.float32, device=dev)
     _need(A_cat, torch.float32, "A_cat", 2)
     _need(B_cat, torch.float32, "B_cat", 2)
+    _shape(A_cat, (R, d_in), "A_cat")
+    _shape(B_cat, (d_out, R), "B_cat")
+    _same_device(A_cat, B_cat, *As, *Bs)
     a_ptrs = (ctypes.c_void_p * n)(*[A.data_ptr() for A in As])
     b_ptrs = (ctypes.c_void_p * n)(*[B.data_ptr() for B in Bs])
     r_arr = (ctypes.c_int * n)(*ranks)
@@ -231,10 +260,12 @@ def lora_linear(x, W, A_cat, B_cat, y=None, workspace=None):
     if y is None:
         y = torch.empty((M, N), dtype=torch.bfloat16, device=x.device)
     _need(y, torch.bfloat16, "y", 2)
+    _shape(y, (M, N), "y")
     need = lora_linear_workspace_size(M, K, N, R)
     if workspace is None and need > 0:
         workspace = torch.empty(need, dtype=torch.uint8, device=x.device)
     ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    _same_device(x, W, A_cat, B_cat, y, workspace)
     with torch.cuda.device(x.device):
         st = lib.lg_lora_linear(_ptr(x), _ptr(W), _ptr(A_cat), _ptr(B_cat), _ptr(y), M, K, N, R,
                                 _ptr(workspace), ws_bytes, _stream(x.device))
@@ -257,6 +288,9 @@ def mx_quantize(x, codes=None, scales=None):
     if scales is None:
         scales = torch.empty(max(mx_scale_bytes(rows, K), 1), dtype=torch.uint8, device=x.device)
     _need(codes, torch.uint8, "codes", 2)
+    _shape(codes, (rows, K), "codes")
+    _at_least(scales, mx_scale_bytes(rows, K), "scales")
+    _same_device(x, codes, scales)
     with torch.cuda.device(x.device):
         st = lib.lg_mx_quantize(_ptr(x), rows, K, _ptr(codes), _ptr(scales), _stream(x.device))
     _check(st, "lg_mx_quantize")
@@ -268,16 +302,11 @@ def lora_linear_mxfp8(x, x_mx, W_mx, A_cat, B_cat, y=None, workspace=None):
     W_mx = mx_quantize(W) (pairs of codes and scales); the LoRA term from the
     bf16 x.  K must be a multiple of 128."""
     _need(x, torch.bfloat16, "x", 2)
-    xq, xsf = x_mx
-    wq, wsf = W_mx
-    _need(xq, torch.uint8, "x codes", 2)
-    _need(wq, torch.uint8, "W codes", 2)
     M, K = x.shape
-    N = wq.shape[0]
-    if tuple(xq.shape) != (M, K) or wq.shape[1] != K:
-        raise ValueError("codes must be [M, K] and [N, K]")
-    if xsf.numel() < mx_scale_bytes(M, K) or wsf.numel() < mx_scale_bytes(N, K):
-        raise ValueError("scale buffers too small")
+    _need(W_mx[0], torch.uint8, "W codes", 2)
+    N = W_mx[0].shape[0]
+    xq, xsf = _scales(x_mx, M, K, "x")
+    wq, wsf = _scales(W_mx, N, K, "W")
     R = 0
     if A_cat is not None and A_cat.numel() > 0:
         _need(A_cat, torch.float32, "A_cat", 2)
@@ -290,10 +319,12 @@ def lora_linear_mxfp8(x, x_mx, W_mx, A_cat, B_cat, y=None, workspace=None):
     if y is None:
         y = torch.empty((M, N), dtype=torch.bfloat16, device=x.device)
     _need(y, torch.bfloat16, "y", 2)
+    _shape(y, (M, N), "y")
     need = lora_linear_workspace_size(M, K, N, R)
     if workspace is None and need > 0:
         workspace = torch.empty(need, dtype=torch.uint8, device=x.device)
     ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    _same_device(x, xq, xsf, wq, wsf, A_cat, B_cat, y, workspace)
     with torch.cuda.device(x.device):
         st = lib.lg_lora_linear_mxfp8(_ptr(x), _ptr(xq), _ptr(xsf), _ptr(wq), _ptr(wsf), _ptr(A_cat), _ptr(B_cat),
                                       _ptr(y), M, K, N, R, _ptr(workspace), ws_bytes, _stream(x.device))
@@ -306,11 +337,14 @@ def lora_linear_swiglu_mxfp8(x, x_mx, W2_mx, A_cat, B_cat, out=None, workspace=N
     (gate rows, then up rows) as mx_quantize(W2); returns (codes [M, F], scales)
     of silu(z[:, :F]) * z[:, F:] with z = x W2^T + LoRA."""
     _need(x, torch.bfloat16, "x", 2)
-    xq, xsf = x_mx
-    wq, wsf = W2_mx
     M, K = x.shape
-    N2 = wq.shape[0]
+    _need(W2_mx[0], torch.uint8, "W2 codes", 2)
+    N2 = W2_mx[0].shape[0]
+    if N2 % 2:
+        raise ValueError("W2 must have 2F rows (gate rows, then up rows)")
     F = N2 // 2
+    xq, xsf = _scales(x_mx, M, K, "x")
+    wq, wsf = _scales(W2_mx, N2, K, "W2")
     R = 0
     if A_cat is not None and A_cat.numel() > 0:
         _need(A_cat, torch.float32, "A_cat", 2)
@@ -323,10 +357,14 @@ def lora_linear_swiglu_mxfp8(x, x_mx, W2_mx, A_cat, B_cat, out=None, workspace=N
     if out is None:
         out = (torch.empty((M, F), dtype=torch.uint8, device=x.device),
                torch.empty(max(mx_scale_bytes(M, F), 1), dtype=torch.uint8, device=x.device))
+    _need(out[0], torch.uint8, "output codes", 2)
+    _shape(out[0], (M, F), "output codes")
+    _at_least(out[1], mx_scale_bytes(M, F), "output scales")
     need = lora_linear_workspace_size(M, K, N2, R)
     if workspace is None and need > 0:
         workspace = torch.empty(need, dtype=torch.uint8, device=x.device)
     ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    _same_device(x, xq, xsf, wq, wsf, A_cat, B_cat, out[0], out[1], workspace)
     with torch.cuda.device(x.device):
         st = lib.lg_lora_linear_swiglu_mxfp8(_ptr(x), _ptr(xq), _ptr(xsf), _ptr(wq), _ptr(wsf), _ptr(A_cat),
                                              _ptr(B_cat), _ptr(out[0]), _ptr(out[1]), M, K, F, R, _ptr(workspace),
@@ -371,6 +409,7 @@ def lora_linear_euler(x, W, A_cat, B_cat, z, sigma, sigma_next, frame_tokens, z_
     if workspace is None and need > 0:
         workspace = torch.empty(need, dtype=torch.uint8, device=x.device)
     ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    _same_device(x, W, A_cat, B_cat, z, z_bf16, workspace)
     with torch.cuda.device(x.device):
         st = lib.lg_lora_linear_euler(_ptr(x), _ptr(W), _ptr(A_cat), _ptr(B_cat), _ptr(z), _ptr(z_bf16), M, K, N, R,
                                       int(frame_tokens), float(sigma), float(sigma_next), _ptr(workspace), ws_bytes,
@@ -388,13 +427,19 @@ def lora_linear_noalloc(x, W, A_cat, B_cat, y):
     _need(y, torch.bfloat16, "y", 2)
     M, K = x.shape
     N = W.shape[0]
+    if W.shape[1] != K:
+        raise ValueError("W must be [N, K]")
+    _shape(y, (M, N), "y")
     R = 0
     if A_cat is not None and A_cat.numel() > 0:
         _need(A_cat, torch.float32, "A_cat", 2)
         _need(B_cat, torch.float32, "B_cat", 2)
         R = A_cat.shape[0]
+        if A_cat.shape[1] != K or tuple(B_cat.shape) != (N, R):
+            raise ValueError("A_cat must be [R, K] and B_cat [N, R]")
     else:
         A_cat = B_cat = None
+    _same_device(x, W, A_cat, B_cat, y)
     with torch.cuda.device(x.device):
         st = lib.lg_lora_linear_noalloc(_ptr(x), _ptr(W), _ptr(A_cat), _ptr(B_cat), _ptr(y), M, K, N, R,
                                         _stream(x.device))
@@ -410,6 +455,7 @@ def renoise(up, sigma, seed, offset=0, out=None):
     _need(out, torch.float32, "out")
     if out.numel() != up.numel():
         raise ValueError("out must have as many elements as up")
+    _same_device(up, out)
     with torch.cuda.device(up.device):
         st = lib.lg_renoise(_ptr(up), _ptr(out), up.numel(), float(sigma), int(seed), int(offset), _stream(up.device))
     _check(st, "lg_renoise")
@@ -422,6 +468,7 @@ def euler_step(x, v, sigma, sigma_next):
     _need(v, torch.float32, "v")
     if x.numel() != v.numel():
         raise ValueError("x and v must have the same number of elements")
+    _same_device(x, v)
     with torch.cuda.device(x.device):
         st = lib.lg_euler_step(_ptr(x), _ptr(v), x.numel(), float(sigma), float(sigma_next), _stream(x.device))
     _check(st, "lg_euler_step")

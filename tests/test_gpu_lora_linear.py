@@ -223,3 +223,26 @@ def test_narrow_n_single_tile(variant, N):
         lg.set_kernel_variant(0)
     assert lg.get_last_device_error() == lg.LG_OK
     assert err <= TOL, err
+
+
+def test_binding_rejects_wrong_output_shapes_before_launch():
+    """The binding checks what the C ABI cannot see (output extents, scale
+    buffer sizes) and raises before any pointer reaches the library."""
+    x, W, A, B = _rand_layer(256, 128, 64, 64, seed=3)
+    n0 = lg.launch_count()
+    with pytest.raises(ValueError):
+        lg.lora_linear(x, W, A, B, y=torch.empty(256, 32, dtype=torch.bfloat16, device=DEV))
+    with pytest.raises(ValueError):
+        lg.lora_linear_noalloc(x, W, A, B, torch.empty(255, 64, dtype=torch.bfloat16, device=DEV))
+    xq, wq = lg.mx_quantize(x), lg.mx_quantize(W)
+    n1 = lg.launch_count()
+    with pytest.raises(ValueError):
+        lg.lora_linear_mxfp8(x, (xq[0], xq[1][:100]), wq, A, B)
+    with pytest.raises(ValueError):
+        lg.mx_quantize(x, codes=torch.empty(256, 64, dtype=torch.uint8, device=DEV))
+    with pytest.raises(ValueError):
+        lg.lora_linear_swiglu_mxfp8(x, xq, wq, A, B, out=(torch.empty(256, 64, dtype=torch.uint8, device=DEV),
+                                                          torch.empty(16, dtype=torch.uint8, device=DEV)))
+    with pytest.raises(ValueError):
+        lg.lora_linear(x, W, A, B.cpu())
+    assert lg.launch_count() == n1 and n1 - n0 == 2
