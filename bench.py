@@ -384,6 +384,28 @@ def run_ic_routes(P, args, world, peaks):
     return out
 
 
+def _time_alternating(f, g, reps, world):
+    """Median ms of f and of g over reps rounds of f then g (one untimed call
+    of each first), CUDA events around every call on the current stream, max
+    over ranks.  Alternating keeps both forms under the same clock and power
+    state."""
+    f()
+    g()
+    torch.cuda.synchronize()
+    barrier(world)
+    tf, tg = [], []
+    for _ in range(reps):
+        for fn, acc in ((f, tf), (g, tg)):
+            e0 = torch.cuda.Event(enable_timing=True)
+            e1 = torch.cuda.Event(enable_timing=True)
+            e0.record()
+            fn()
+            e1.record()
+            torch.cuda.synchronize()
+            acc.append(e0.elapsed_time(e1))
+    return max_over_ranks(statistics.median(tf), world), max_over_ranks(statistics.median(tg), world)
+
+
 def run_fusions(P, args, world, peaks):
     """Epilogue fusions beside the step, each against its unfused form:
 
@@ -396,12 +418,13 @@ def run_fusions(P, args, world, peaks):
       MXFP8 quantizer fused (lg_lora_linear_swiglu_mxfp8) on a quarter of the
       tokens (the unfused form holds the [M, 2 ffn] intermediate); unfused:
       lg_lora_linear_mxfp8, torch silu(gate) * up in bf16, lg_mx_quantize.
+    Fused and unfused calls alternate; each figure is a median.
     """
     import lora_gemm_b200 as lg
     from lora_gemm_b200 import synth
 
     w, dev, R = P.w, P.up.device, P.R
-    reps = max(args.steps, 2)
+    reps = max(args.steps, 5)
     out = {}
     L0 = P.layers[0]
     K = L0["K"]
@@ -419,8 +442,6 @@ def run_fusions(P, args, world, peaks):
         zb = torch.empty_like(z, dtype=torch.bfloat16)
         ws = torch.empty(lg.lora_linear_euler_workspace_size(M, K, C, R), dtype=torch.uint8, device=dev)
         s0, s1 = P.sigmas[1], P.sigmas[2]
-        fused_ms = _time_calls(lambda: lg.lora_linear_euler(x, W, A_cat, B_cat, z, s0, s1, T, z_bf16=zb,
-                                                            workspace=ws), reps, world)
         Cp = 32
         Wp = torch.zeros((Cp, K), dtype=torch.bfloat16, device=dev)
         Wp[:C] = W
@@ -435,7 +456,9 @@ def run_fusions(P, args, world, peaks):
             lg.euler_step(z, v, s0, s1)
             zb.copy_(z)
 
-        unfused_ms = _time_calls(unfused, reps, world)
+        fused_ms, unfused_ms = _time_alternating(
+            lambda: lg.lora_linear_euler(x, W, A_cat, B_cat, z, s0, s1, T, z_bf16=zb, workspace=ws), unfused,
+            reps, world)
         fl = layer_flops(M, K, C, R)
         peak = peaks["bf16_tflops_sustained"]
         out["projection_euler"] = {
@@ -464,8 +487,6 @@ def run_fusions(P, args, world, peaks):
         q = (torch.empty((Mq, F), dtype=torch.uint8, device=dev),
              torch.empty(lg.mx_scale_bytes(Mq, F), dtype=torch.uint8, device=dev))
         ws = torch.empty(lg.lora_linear_workspace_size(Mq, Km, N2, R), dtype=torch.uint8, device=dev)
-        fused_ms = _time_calls(lambda: lg.lora_linear_swiglu_mxfp8(x, xq, wq, A_cat, B_cat, out=q, workspace=ws),
-                               reps, world)
         y = torch.empty((Mq, N2), dtype=torch.bfloat16, device=dev)
 
         def unfused():
@@ -473,7 +494,8 @@ def run_fusions(P, args, world, peaks):
             s = torch.nn.functional.silu(y[:, :F]) * y[:, F:]
             lg.mx_quantize(s, codes=q[0], scales=q[1])
 
-        unfused_ms = _time_calls(unfused, reps, world)
+        fused_ms, unfused_ms = _time_alternating(
+            lambda: lg.lora_linear_swiglu_mxfp8(x, xq, wq, A_cat, B_cat, out=q, workspace=ws), unfused, reps, world)
         fl = layer_flops(Mq, Km, N2, R)
         peak = 2.0 * peaks["bf16_tflops_sustained"]
         out["swiglu_mxfp8"] = {
