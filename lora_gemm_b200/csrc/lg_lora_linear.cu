@@ -116,6 +116,10 @@ struct Cfg {
   static constexpr uint32_t STAGE = A_BYTES + B_BYTES + (MX ? 2048u : 0u);
   static constexpr int MMA_M = PAIR ? 2 * BM : BM;
   static constexpr int PANEL = PAIR ? 2 * BM : BM;
+  // Folded base term (narrow single-tile layers): its accumulator sits after
+  // the widest down-projection chunk, below h.
+  static constexpr uint32_t Y_FOLD_COL = (uint32_t)HC_MAX;
+  static constexpr int FOLD_MAX_N = BN - HC_MAX;
   static_assert(!MX || PAIR, "the MXFP8 base term runs on SM pairs only");
   static_assert(STAGE % 1024 == 0, "stages must stay 1024-byte aligned");
   static_assert((PAIR ? HC_MAX / 2 : HC_MAX) * BK * 2 <= B_BYTES, "A_cat chunk tile must fit the B slot");
@@ -167,6 +171,10 @@ struct Args {
   // MMA N of the output tiles: BN, or N rounded up to 16 when one tile
   // covers all N columns (the rest of the tile would be zeros); bf16 only.
   int y_n;
+  // 1: the base term x W^T (one tile of y_n <= FOLD_MAX_N columns) is computed
+  // in the first down-projection sweep, from the same x stages, into TMEM
+  // columns Y_FOLD_COL..; phase B then only adds the up-projection.
+  int fold;
   // Euler output (bf16 variants, eu_z != null): v = the FP32 accumulator
   // is not stored; token m's channel c updates the latent z [M / eu_frame, N,
   // eu_frame] in place, z += eu_dt v, and eu_zb (if not null) receives the
@@ -264,6 +272,10 @@ __device__ void run_producer(const CUtensorMap* tm_x, const CUtensorMap* tm_w, c
   const uint32_t a_rows = PAIR ? (uint32_t)a.chunk_n / 2 : (uint32_t)a.chunk_n;
   const uint32_t mult = PAIR ? 2u : 1u;
   const uint32_t tx_a = mult * (A_BYTES + a_rows * BK * 2);
+  // Folded base term: the first sweep's stages also carry y_n W rows (an SM
+  // pair: y_n / 2 per CTA) after the A_cat chunk rows.
+  const uint32_t wf_rows = PAIR ? (uint32_t)a.y_n / 2 : (uint32_t)a.y_n;
+  const uint32_t tx_fold = tx_a + (a.fold ? mult * wf_rows * BK * 2 : 0u);
   const uint32_t tx_k = mult * (A_BYTES + C::B_BYTES + (MX ? 3 * SF_GROUP_BYTES : 0u));
   const uint32_t tx_r = mult * C::B_BYTES;
   uint32_t stage = 0, phase = 0, sweep = 0, it = 0;
@@ -298,9 +310,11 @@ __device__ void run_producer(const CUtensorMap* tm_x, const CUtensorMap* tm_w, c
           break;
         }
         const uint32_t sa = smem_base + stage * C::STAGE;
-        if (posts_tx) mbar_arrive_expect_tx(full_local + 8 * stage, tx_a);
+        const bool fold = a.fold && j == 0;
+        if (posts_tx) mbar_arrive_expect_tx(full_local + 8 * stage, fold ? tx_fold : tx_a);
         load_x(tm_x, sa, kb * BK, m0);
         load(tm_a, sa + A_BYTES, kb * BK, first + half * (int)a_rows);
+        if (fold) load(tm_w, sa + A_BYTES + a_rows * BK * 2, kb * BK, half * (int)wf_rows);
         ++fills;
         advance(stage, phase, stages);
       }
@@ -315,7 +329,7 @@ __device__ void run_producer(const CUtensorMap* tm_x, const CUtensorMap* tm_w, c
     for (int t = member; ok && t < a.n_tiles; t += a.group, ++sweep) {
       // A pair's MMA takes y_n / 2 B rows from each CTA (B_ROWS when y_n = BN).
       const int n0 = a.ffn > 0 ? (half ? a.ffn : 0) + t * BM : t * C::BN + half * (a.y_n / 2);
-      const int kloop = MX ? a.kq_blocks : a.k_blocks;
+      const int kloop = a.fold ? 0 : (MX ? a.kq_blocks : a.k_blocks);
       for (int i = 0; i < kloop; ++i) {
         const int kb = (sweep & 1) ? kloop - 1 - i : i;
         if (!wait_bounded(empty0 + 8 * stage, phase ^ 1, a.wait_limit_ns, abort_flag)) {
@@ -404,13 +418,23 @@ __device__ void run_mma(const Args& a, Control* ctl, uint32_t smem_base, uint32_
       umma_ss(d_acc, da, db, idesc, acc);
     }
   };
-  auto mma_ts = [&](uint32_t a_tmem, uint64_t db) {
+  auto mma_ss_to = [&](uint32_t d, uint64_t da, uint64_t db, uint32_t idesc, uint32_t acc) {
     if constexpr (PAIR) {
-      umma_ts_pair(d_acc, a_tmem, db, idesc_y, 1u);
+      umma_ss_pair(d, da, db, idesc, acc);
     } else {
-      umma_ts(d_acc, a_tmem, db, idesc_y, 1u);
+      umma_ss(d, da, db, idesc, acc);
     }
   };
+  // The output tile's accumulator: the folded one, or the shared region.
+  const uint32_t d_y = a.fold ? tmem + C::Y_FOLD_COL : d_acc;
+  auto mma_ts = [&](uint32_t a_tmem, uint64_t db) {
+    if constexpr (PAIR) {
+      umma_ts_pair(d_y, a_tmem, db, idesc_y, 1u);
+    } else {
+      umma_ts(d_y, a_tmem, db, idesc_y, 1u);
+    }
+  };
+  const uint32_t a_rows = PAIR ? (uint32_t)a.chunk_n / 2 : (uint32_t)a.chunk_n;
   for (int p = (int)cid; ok && p < a.num_panels; p += (int)ncl) {
     for (int j = 0; ok && j < a.n_chunks; ++j) {
       if (!wait_bounded(acc_empty, acc_phase ^ 1, a.wait_limit_ns, abort_flag, PAIR)) {
@@ -429,6 +453,12 @@ __device__ void run_mma(const Args& a, Control* ctl, uint32_t smem_base, uint32_
         const uint64_t db = sw128_kmajor_desc(sa + A_BYTES);
 #pragma unroll
         for (int kk = 0; kk < BK / 16; ++kk) mma_ss(da + 2 * kk, db + 2 * kk, idesc_h, (i | kk) != 0);
+        if (a.fold && j == 0) {
+          // The base term from the same x stage: B = the W rows behind the chunk rows.
+          const uint64_t dw = sw128_kmajor_desc(sa + A_BYTES + a_rows * BK * 2);
+#pragma unroll
+          for (int kk = 0; kk < BK / 16; ++kk) mma_ss_to(d_y, da + 2 * kk, dw + 2 * kk, idesc_y, (i | kk) != 0);
+        }
         commit(empty0 + 8 * stage);
         advance(stage, phase, stages);
       }
@@ -442,7 +472,7 @@ __device__ void run_mma(const Args& a, Control* ctl, uint32_t smem_base, uint32_
         break;
       }
       tc_fence_after();
-      const int kloop = MX ? a.kq_blocks : a.k_blocks;
+      const int kloop = a.fold ? 0 : (MX ? a.kq_blocks : a.k_blocks);
       for (int i = 0; i < kloop; ++i) {
         if (!wait_bounded(full0 + 8 * stage, phase, a.wait_limit_ns, abort_flag)) {
           ok = false;
@@ -494,7 +524,7 @@ __device__ void run_mma(const Args& a, Control* ctl, uint32_t smem_base, uint32_
           const uint64_t dh =
               sw128_kmajor_desc(smem_base + a.h_tile_off + (uint32_t)(rb * BK - C::R_TMEM) / BK * H_TILE_BYTES);
 #pragma unroll
-          for (int kk = 0; kk < BK / 16; ++kk) mma_ss(dh + 2 * kk, db + 2 * kk, idesc_y, 1u);
+          for (int kk = 0; kk < BK / 16; ++kk) mma_ss_to(d_y, dh + 2 * kk, db + 2 * kk, idesc_y, 1u);
         }
         commit(empty0 + 8 * stage);
         advance(stage, phase, stages);
@@ -803,6 +833,8 @@ __device__ void run_epilogue(const CUtensorMap* tm_y, const Args& a, Control* ct
       }
       release_acc(true);
     }
+    // The output tile's accumulator columns (folded base term: Y_FOLD_COL..).
+    const uint32_t y_col = a.fold ? C::Y_FOLD_COL : ACC_COL;
     for (int t = member; ok && t < a.n_tiles; t += a.group) {
       ok = __all_sync(0xffffffffu, wait_bounded(acc_full, acc_phase, a.wait_limit_ns, abort_flag));
       if (!ok) break;
@@ -831,7 +863,7 @@ __device__ void run_epilogue(const CUtensorMap* tm_y, const Args& a, Control* ct
           // handed back before the stores; wider tiles are stored 16 columns
           // at a time and hand it back at the end.
           const int cols = a.y_n / 2;
-          const uint32_t src = lane_base + ACC_COL + (uint32_t)(half * cols);
+          const uint32_t src = lane_base + y_col + (uint32_t)(half * cols);
           const int col0 = t * C::BN + half * cols;
           const int64_t row = m0 + row_in_tile;
           if (cols <= 32) {
@@ -858,7 +890,7 @@ __device__ void run_epilogue(const CUtensorMap* tm_y, const Args& a, Control* ct
       // conversion and the stores below.
       constexpr int N32 = C::HALF_N / 32;
       constexpr bool TAIL16 = (C::HALF_N % 32) != 0;
-      const uint32_t src = lane_base + ACC_COL + (uint32_t)(half * C::HALF_N);
+      const uint32_t src = lane_base + y_col + (uint32_t)(half * C::HALF_N);
       uint32_t v[N32 + (TAIL16 ? 1 : 0)][32];
 #pragma unroll
       for (int i = 0; i < N32; ++i) tmem_ld_32x32b_x32(src + 32 * i, v[i]);
@@ -1185,6 +1217,14 @@ cudaError_t launch_variant(const LinearLaunch& p, cudaStream_t s, int dev, int c
   Geometry geo;
   if (!make_geometry<PAIR, MX>(group, p.R, &geo)) return cudaErrorInvalidConfiguration;
   const uint32_t a_rows = PAIR ? (uint32_t)geo.chunk_n / 2 : (uint32_t)geo.chunk_n;
+  const int n_tiles = p.ffn > 0 ? p.ffn / BM : (p.N + C::BN - 1) / C::BN;
+  const int y_n = (!MX && n_tiles == 1) ? (p.N + 15) / 16 * 16 : C::BN;
+  // Fold the base term into the first down-projection sweep when the layer is
+  // one narrow tile: its W rows then fit beside the chunk rows of A_cat in
+  // the stage, and its accumulator beside the chunk's in TMEM.
+  const uint32_t wf_rows = PAIR ? (uint32_t)y_n / 2 : (uint32_t)y_n;
+  const bool fold = !MX && p.R > 0 && group == 1 && n_tiles == 1 && y_n <= C::FOLD_MAX_N &&
+                    (a_rows + wf_rows) * BK * 2 <= C::B_BYTES;
   CUtensorMap tm_x, tm_w, tm_a, tm_b, tm_y, tm_xq, tm_sfa, tm_sfb;
   bool ok = make_map(enc, &tm_x, p.x, (uint64_t)p.K, (uint64_t)p.M, BM);
   if (MX) {
@@ -1195,7 +1235,7 @@ cudaError_t launch_variant(const LinearLaunch& p, cudaStream_t s, int dev, int c
          make_map_scales(enc, &tm_sfa, p.xsf, (uint64_t)((p.M + BM - 1) / BM) * kg) &&
          make_map_scales(enc, &tm_sfb, p.wsf, (uint64_t)((p.N + BM - 1) / BM) * kg);
   } else {
-    ok = ok && make_map(enc, &tm_w, p.W, (uint64_t)p.K, (uint64_t)p.N, C::B_ROWS);
+    ok = ok && make_map(enc, &tm_w, p.W, (uint64_t)p.K, (uint64_t)p.N, fold ? wf_rows : C::B_ROWS);
     tm_xq = tm_x;  // never read without MXFP8
     tm_sfa = tm_x;
     tm_sfb = tm_x;
@@ -1226,9 +1266,10 @@ cudaError_t launch_variant(const LinearLaunch& p, cudaStream_t s, int dev, int c
   args.N = p.N;
   args.R = p.R;
   args.num_panels = (int)((p.M + C::PANEL - 1) / C::PANEL);
-  args.n_tiles = p.ffn > 0 ? p.ffn / BM : (p.N + C::BN - 1) / C::BN;
+  args.n_tiles = n_tiles;
   args.ffn = p.ffn;
-  args.y_n = (!MX && args.n_tiles == 1) ? (p.N + 15) / 16 * 16 : C::BN;
+  args.y_n = y_n;
+  args.fold = fold ? 1 : 0;
   args.eu_z = p.eu_z;
   args.eu_zb = reinterpret_cast<uint16_t*>(p.eu_zb);
   args.eu_frame = p.eu_frame;

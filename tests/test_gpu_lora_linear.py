@@ -210,7 +210,7 @@ def test_cluster_size_argument_checked():
 
 
 @pytest.mark.parametrize("variant", [1, 2])
-@pytest.mark.parametrize("N", [32, 96, 160, 224])
+@pytest.mark.parametrize("N", [32, 64, 96, 160, 224])
 def test_narrow_n_single_tile(variant, N):
     """N below the tile width: one output tile whose MMAs run with N columns
     (an SM pair takes N / 2 B rows from each CTA)."""
