@@ -339,6 +339,47 @@ def _time_calls(fn, reps, world):
     return max_over_ranks(t0.elapsed_time(t1) / reps, world)
 
 
+def run_elementwise_isolated(P, args, world, peaks):
+    """renoise and euler_step timed alone: 100 back-to-back launches each,
+    rotating over 4 buffer sets (408 MB, more than L2 holds), CUDA events
+    around the whole loop.  The in-step figures come from the bench step."""
+    import lora_gemm_b200 as lg
+
+    hbm = peaks["hbm_gbs"]
+    n = P.up.numel()
+    sets = 4
+    ups = [P.up.clone() for _ in range(sets)]
+    xs = [torch.empty_like(P.up) for _ in range(sets)]
+    vs = [P.v[i % len(P.v)].clone() for i in range(sets)]
+    s0, s1 = P.sigmas[0], P.sigmas[1]
+    out = {}
+    for name, per_elem, fn in (
+            ("renoise", 8.0, lambda i: lg.renoise(ups[i], s0, P.w.seed, offset=P.noise_offset, out=xs[i])),
+            ("euler_step", 12.0, lambda i: lg.euler_step(xs[i], vs[i], s0, s1))):
+        for i in range(sets):
+            fn(i)
+        torch.cuda.synchronize()
+        barrier(world)
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        launches = 100
+        e0.record()
+        for k in range(launches):
+            fn(k % sets)
+        e1.record()
+        torch.cuda.synchronize()
+        ms = max_over_ranks(e0.elapsed_time(e1) / launches, world)
+        gbs = per_elem * n / (ms * 1e-3) / 1e9
+        out[name] = {"launches": launches, "ms": round(ms, 5), "gbs": round(gbs, 1),
+                     "frac_of_measured_hbm": round(gbs / hbm, 4)}
+    out["note"] = f"{sets} rotating buffer sets ({sets * 2 * 4 * n / 1e6:.0f} MB) so that no launch finds its data in L2"
+    del ups, xs, vs
+    status = lg.get_last_device_error()
+    if status != lg.LG_OK:
+        raise SystemExit(f"device error during the isolated elementwise runs: {lg.status_string(status)}")
+    return out
+
+
 def run_ic_routes(P, args, world, peaks):
     """The IC sampler routes (up3, up4, hf8: re-noise at the route's start and
     one Euler step per rung of HyperFlow's shift-12 ladder) on the workload's
@@ -653,6 +694,7 @@ def run_ours(args, rank, world, local):
     if not args.no_fusions:
         result["fusions"] = run_fusions(P, args, world, peaks)
         result["ic_routes"] = run_ic_routes(P, args, world, peaks)
+        result["elementwise_isolated"] = run_elementwise_isolated(P, args, world, peaks)
     if not args.no_e2e:
         result["e2e"] = run_e2e(P, args, world)
     if rank == 0 and not args.no_cpu_baseline:
@@ -936,7 +978,7 @@ def main():
     ap.add_argument("--workload", default=WORKLOAD)
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-mxfp8", action="store_true")
-    ap.add_argument("--no-fusions", action="store_true", help="skip the fused-epilogue comparisons and the IC routes")
+    ap.add_argument("--no-fusions", action="store_true", help="skip the fused-epilogue comparisons, the IC routes and the isolated elementwise runs")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--tokens", type=int, default=None,
