@@ -131,3 +131,60 @@ def test_host_validation_merge():
     assert L.lg_lora_merge(3, ptrs, bptrs, ranks, scales, 66, 64, Ac, Bc, None) == lg.LG_ERR_UNSUPPORTED_SHAPE
     assert L.lg_lora_merge(3, ptrs, bptrs, ranks, scales, 64, 64, MIS, Bc, None) == lg.LG_ERR_MISALIGNED
     assert L.lg_lora_merge(3, ptrs, bptrs, ranks, scales, 64, 64, None, Bc, None) == lg.LG_ERR_INVALID_ARG
+
+
+def test_host_validation_fused_and_mxfp8_entry_points():
+    """Argument checks of the MXFP8, SwiGLU and Euler entry points run before
+    anything touches a device (fake pointers, no GPU needed)."""
+    import lora_gemm_b200 as lg
+
+    L = lg.lib
+    ws, out, sc = P(0x7F0040000000), P(0x7F0080000000), P(0x7F00C0000000)
+    xq, xs, wq, wsf = P(0x7F0100000000), P(0x7F0140000000), P(0x7F0180000000), P(0x7F01C0000000)
+    A, B = P(0x7F0010000000), P(0x7F0020000000)
+    big = 1 << 30
+
+    def mx(M=256, K=128, N=128, R=64, x=A16, y=out, ws_bytes=big, xq=xq):
+        return L.lg_lora_linear_mxfp8(x, xq, xs, wq, wsf, A, B, y, M, K, N, R, ws, ws_bytes, None)
+
+    assert mx(K=192) == lg.LG_ERR_UNSUPPORTED_SHAPE          # K not a multiple of 128
+    assert mx(N=48) == lg.LG_ERR_UNSUPPORTED_SHAPE
+    assert mx(xq=None) == lg.LG_ERR_INVALID_ARG
+    assert mx(xq=MIS) == lg.LG_ERR_MISALIGNED
+    assert mx(y=P(xq.value + 1024)) == lg.LG_ERR_INVALID_ARG  # y overlaps the x codes
+    assert mx(ws_bytes=0) == lg.LG_ERR_WORKSPACE
+    assert mx(M=0) == lg.LG_OK
+
+    def sw(M=256, K=128, F=128, R=64, codes=out, scales=sc):
+        return L.lg_lora_linear_swiglu_mxfp8(A16, xq, xs, wq, wsf, A, B, codes, scales, M, K, F, R, ws, big, None)
+
+    assert sw(F=96) == lg.LG_ERR_UNSUPPORTED_SHAPE           # F not a multiple of 128
+    assert sw(codes=None) == lg.LG_ERR_INVALID_ARG
+    assert sw(scales=MIS) == lg.LG_ERR_MISALIGNED
+    assert sw(scales=P(out.value + 64)) == lg.LG_ERR_INVALID_ARG  # scales overlap the codes
+    assert sw(M=0) == lg.LG_OK
+
+    def eu(M=256, K=128, N=24, R=64, z=out, zb=sc, T=128, s0=0.857, s1=0.667, ws_bytes=big):
+        return L.lg_lora_linear_euler(A16, A16b, A, B, z, zb, M, K, N, R, T, s0, s1, ws, ws_bytes, None)
+
+    assert eu(N=0) == lg.LG_ERR_UNSUPPORTED_SHAPE
+    assert eu(K=96) == lg.LG_ERR_UNSUPPORTED_SHAPE
+    assert eu(T=100) == lg.LG_ERR_INVALID_ARG                 # M not a multiple of the frame
+    assert eu(T=0) == lg.LG_ERR_INVALID_ARG
+    assert eu(s1=float("nan")) == lg.LG_ERR_INVALID_ARG
+    assert eu(z=None) == lg.LG_ERR_INVALID_ARG
+    assert eu(z=MIS) == lg.LG_ERR_MISALIGNED
+    assert eu(zb=P(out.value + 256)) == lg.LG_ERR_INVALID_ARG  # bf16 copy overlaps z
+    assert eu(z=P(A16.value + 256)) == lg.LG_ERR_INVALID_ARG   # z overlaps x
+    assert eu(ws_bytes=16) == lg.LG_ERR_WORKSPACE
+    assert eu(M=0) == lg.LG_OK
+    assert eu(M=0, zb=None) == lg.LG_OK
+
+    def a256(v):
+        return (v + 255) // 256 * 256
+
+    assert lg.lora_linear_euler_workspace_size(532800, 7168, 24, 576) == a256(2 * 576 * 7168) + a256(2 * 24 * 576)
+    assert lg.lora_linear_euler_workspace_size(10, 7168, 24, 0) == 0
+    assert lg.lora_linear_euler_workspace_size(10, 100, 24, 64) == 0
+    assert L.lg_mx_quantize(None, 4, 128, out, sc, None) == lg.LG_ERR_INVALID_ARG
+    assert L.lg_mx_quantize(A16, 4, 96, out, sc, None) == lg.LG_ERR_UNSUPPORTED_SHAPE
