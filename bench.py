@@ -697,6 +697,8 @@ def run_ours(args, rank, world, local):
         result["elementwise_isolated"] = run_elementwise_isolated(P, args, world, peaks)
     if not args.no_e2e:
         result["e2e"] = run_e2e(P, args, world)
+        # Hand the pinned buffers back to the host (torch keeps them cached).
+        torch._C._host_emptyCache()
     if rank == 0 and not args.no_cpu_baseline:
         result["cpu_baseline"] = cpu_baseline(w, target_s=args.cpu_seconds)
     return result
@@ -754,13 +756,47 @@ def run_e2e(P, args, world):
         if last_use[id(L["x"])] == k:
             inputs.append(L["x"])
         inputs.append(P.v[k])
-    host_in = {id(t): pinned(t) for t in inputs}
     outputs = [L["y"] for L in P.layers] + [P.x_lat]
-    host_out = {id(t): pinned(t) for t in outputs}
-    for t in inputs:
-        host_in[id(t)].copy_(t)
     h2d = sum(t.numel() * t.element_size() for t in inputs)
     d2h = sum(t.numel() * t.element_size() for t in outputs)
+
+    # Pinned host buffers, within this rank's share of the host's memory (the
+    # ranks of a node share it): separate input and output buffers when they
+    # fit, else one pool that the outputs overwrite after the inputs were read
+    # from it (same copies, same timing; later steps then read back earlier
+    # results as their inputs), else no end-to-end figure.
+    def padded(t):
+        return (t.numel() * t.element_size() + 4095) // 4096 * 4096
+
+    need_in, need_out = sum(padded(t) for t in inputs), sum(padded(t) for t in outputs)
+    # Every rank reads the free memory before any rank pins, and all take the
+    # most restrictive choice, so that they run the same collectives.
+    barrier(world)
+    budget = _host_budget()
+    choice = 0 if budget is None or need_in + need_out <= budget else (1 if max(need_in, need_out) <= budget else 2)
+    choice = int(max_over_ranks(float(choice), world))
+    if choice == 0:
+        host_mode = "separate"
+        host_in = {id(t): pinned(t) for t in inputs}
+        host_out = {id(t): pinned(t) for t in outputs}
+    elif choice == 1:
+        host_mode = "shared pool (host memory)"
+        pool = torch.empty(max(need_in, need_out), dtype=torch.uint8, pin_memory=True)
+
+        def carve(ts):
+            views, off = {}, 0
+            for t in ts:
+                n = t.numel() * t.element_size()
+                views[id(t)] = pool[off:off + n].view(t.dtype).view(t.shape)
+                off += padded(t)
+            return views
+
+        host_in, host_out = carve(inputs), carve(outputs)
+    else:
+        return {"unavailable": f"host memory: the step's pinned buffers need {max(need_in, need_out) / 1e9:.0f} GB "
+                               "per rank even shared, more than a rank's share of the node's free memory"}
+    for t in inputs:
+        host_in[id(t)].copy_(t)
 
     arrived = {}    # input -> event: this step's copy-in is done
     released = {}   # input -> event: the previous step's last use of its device buffer is done
@@ -847,8 +883,20 @@ def run_e2e(P, args, world):
             raise RuntimeError("e2e: a copied-out result differs from the device result")
     return {"value": round(_dist().whole_job_rate(P.M, world, steps, ms), 1), "unit": UNIT,
             "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h), "steps": steps,
-            "ms_per_step": round(ms / steps, 3),
+            "ms_per_step": round(ms / steps, 3), "host_buffers": host_mode,
             "overlap": "host->device, compute and device->host on three streams, ordered by events per buffer"}
+
+
+def _host_budget():
+    """Bytes of host memory this rank may pin: 80 % of what the kernel reports
+    available, split among the ranks of this node; None if unknown."""
+    try:
+        with open("/proc/meminfo") as f:
+            avail = next(int(line.split()[1]) * 1024 for line in f if line.startswith("MemAvailable"))
+    except (OSError, StopIteration, ValueError):
+        return None
+    local = int(os.environ.get("LOCAL_WORLD_SIZE", "1") or 1)
+    return 0.8 * avail / max(local, 1)
 
 
 # ---------------------------------------------------------------------------
