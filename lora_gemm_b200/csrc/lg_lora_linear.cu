@@ -39,6 +39,11 @@
 //     allocation, warps 2-9 are the epilogue: each pulls half of the tile's
 //     accumulator into registers, releases the TMEM accumulator to the next
 //     tile's MMAs, then converts and stores y.
+//   * Output variants: bf16 y (the default); the FP32 latent updated in place
+//     by an Euler step (eu_z); MXFP8 codes and scales of silu(gate) * up
+//     (ffn, MXFP8 base term only).  A layer of one narrow tile (fold)
+//     computes its base term in the first down-projection sweep, from the
+//     same x stages, instead of sweeping x once more in phase B.
 //   * Every mbarrier wait is bounded; on expiry the kernel records
 //     LG_ERR_DEVICE_TIMEOUT in the device error word, drains its own TMA
 //     copies and MMAs, frees its TMEM and returns.
