@@ -211,9 +211,13 @@ def run_step(P, ev=None):
     for L in P.layers:
         rec("lora_merge", lambda L=L: lg.lora_merge(L["As"], L["Bs"], P.scales, L["A_cat"], L["B_cat"]))
     rec("renoise", lambda: lg.renoise(P.up, P.sigmas[0], P.w.seed, offset=P.noise_offset, out=P.x_lat))
-    for k, L in enumerate(P.layers):
-        rec(f"lora_linear{k}", lambda L=L: lg.lora_linear(L["x"], L["W"], L["A_cat"], L["B_cat"], y=L["y"],
-                                                          workspace=L["ws"]))
+    # Euler step k follows layer k; a workload with fewer layers than steps
+    # (768P, tiny: one layer) runs the remaining steps after it.
+    for k in range(len(P.sigmas) - 1):
+        if k < len(P.layers):
+            L = P.layers[k]
+            rec(f"lora_linear{k}", lambda L=L: lg.lora_linear(L["x"], L["W"], L["A_cat"], L["B_cat"], y=L["y"],
+                                                              workspace=L["ws"]))
         rec(f"euler{k}", lambda k=k: lg.euler_step(P.x_lat, P.v[k], P.sigmas[k], P.sigmas[k + 1]))
 
 
@@ -248,12 +252,14 @@ def run_mxfp8(P, args, world, peaks):
         for L in P.layers:
             rec("lora_merge", lambda L=L: lg.lora_merge(L["As"], L["Bs"], P.scales, L["A_cat"], L["B_cat"]))
         rec("renoise", lambda: lg.renoise(P.up, P.sigmas[0], P.w.seed, offset=P.noise_offset, out=P.x_lat))
-        for k, L in enumerate(P.layers):
-            if first_use[id(L["x"])] == k:
-                q = xq[id(L["x"])]
-                rec("quantize", lambda L=L, q=q: lg.mx_quantize(L["x"], codes=q[0], scales=q[1]))
-            rec(f"lin{k}", lambda k=k, L=L: lg.lora_linear_mxfp8(L["x"], xq[id(L["x"])], wq[k], L["A_cat"], L["B_cat"],
-                                                                  y=L["y"], workspace=L["ws"]))
+        for k in range(len(P.sigmas) - 1):
+            if k < len(P.layers):
+                L = P.layers[k]
+                if first_use[id(L["x"])] == k:
+                    q = xq[id(L["x"])]
+                    rec("quantize", lambda L=L, q=q: lg.mx_quantize(L["x"], codes=q[0], scales=q[1]))
+                rec(f"lin{k}", lambda k=k, L=L: lg.lora_linear_mxfp8(L["x"], xq[id(L["x"])], wq[k], L["A_cat"],
+                                                                      L["B_cat"], y=L["y"], workspace=L["ws"]))
             rec(f"euler{k}", lambda k=k: lg.euler_step(P.x_lat, P.v[k], P.sigmas[k], P.sigmas[k + 1]))
 
     for _ in range(max(args.warmup, 1)):
@@ -616,7 +622,7 @@ def run_ours(args, rank, world, local):
     lin_ms = [statistics.mean(per[f"lora_linear{k}"]) for k in range(len(P.layers))]
     achieved_tflops = sum(flops) / (sum(lin_ms) * 1e-3) / 1e12
     peak_t = peaks["bf16_tflops_sustained"]
-    traffic = load_traffic()
+    traffic = load_traffic(w.name, M)
     bpk = bytes_per_kernel(P)
     ren_ms = statistics.mean(per["renoise"])
     eul_ms = statistics.mean([t for k in range(3) for t in per[f"euler{k}"]])
@@ -704,9 +710,10 @@ def run_ours(args, rank, world, local):
     return result
 
 
-def load_traffic():
+def load_traffic(workload, tokens):
     """DRAM bytes per lora_linear launch from the committed ncu summary, or None
-    when the summary is missing or was taken on a different kernel source."""
+    when the summary is missing, was taken on a different kernel source, or
+    was scaled to another workload or token count."""
     import hashlib
 
     path = os.path.join(ROOT, "profiles", "lora_linear_traffic.json")
@@ -718,7 +725,7 @@ def load_traffic():
             digest = hashlib.sha256(f.read()).hexdigest()
     except (OSError, ValueError):
         return None
-    if t.get("kernel_source_sha256") != digest:
+    if t.get("kernel_source_sha256") != digest or workload != "2k" or t.get("scaled_to_tokens") != tokens:
         return None
     return t.get("traffic_bytes_per_launch")
 
@@ -752,9 +759,9 @@ def run_e2e(P, args, world):
     for k, L in enumerate(P.layers):
         last_use[id(L["x"])] = k
     inputs = [P.up]
-    for k, L in enumerate(P.layers):
-        if last_use[id(L["x"])] == k:
-            inputs.append(L["x"])
+    for k in range(len(P.sigmas) - 1):
+        if k < len(P.layers) and last_use[id(P.layers[k]["x"])] == k:
+            inputs.append(P.layers[k]["x"])
         inputs.append(P.v[k])
     outputs = [L["y"] for L in P.layers] + [P.x_lat]
     h2d = sum(t.numel() * t.element_size() for t in inputs)
@@ -841,13 +848,15 @@ def run_e2e(P, args, world):
         write(P.x_lat)
         lg.renoise(up, P.sigmas[0], P.w.seed, offset=P.noise_offset, out=P.x_lat)
         release(P.up)
-        for k, L in enumerate(P.layers):
-            x = use(L["x"])
-            write(L["y"])
-            lg.lora_linear(x, L["W"], L["A_cat"], L["B_cat"], y=L["y"], workspace=L["ws"])
-            if last_use[id(L["x"])] == k:
-                release(L["x"])
-            copy_out(L["y"])
+        for k in range(len(P.sigmas) - 1):
+            if k < len(P.layers):
+                L = P.layers[k]
+                x = use(L["x"])
+                write(L["y"])
+                lg.lora_linear(x, L["W"], L["A_cat"], L["B_cat"], y=L["y"], workspace=L["ws"])
+                if last_use[id(L["x"])] == k:
+                    release(L["x"])
+                copy_out(L["y"])
             v = use(P.v[k])
             lg.euler_step(P.x_lat, v, P.sigmas[k], P.sigmas[k + 1])
             release(P.v[k])
