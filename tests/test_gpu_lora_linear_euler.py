@@ -59,6 +59,9 @@ def _check(x, W, A, B, R, z_old, z_new, zb, T, s0=S0, s1=S1):
         (2, 333, 100, 256, 128),    # > 32 columns per warp: stored 16 at a time
         (1, 512, 300, 256, 64),     # two N tiles (single-SM; one 256-column pair tile)
         (2, 400, 500, 256, 64),     # two N tiles on either variant
+        (256, 1, 24, 128, 64),      # one cell per frame: the latent is token-major
+        (1, 128, 24, 64, 64),       # smallest K
+        (1, 1, 16, 128, 0),         # a single token
     ],
 )
 @pytest.mark.parametrize("variant", [1, 2])

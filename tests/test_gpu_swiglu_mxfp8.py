@@ -73,6 +73,7 @@ def _check(x, W2, A, B, R, codes, scales):
     "M,K,F,R",
     [
         (256, 128, 128, 0),      # one tile, no LoRA
+        (1, 128, 128, 0),        # a single token (rows 1-127 of the scale group padded with 0)
         (517, 384, 256, 576),    # ragged M, full rank
         (1000, 1024, 512, 64),
         (2304, 1024, 1024, 576),
