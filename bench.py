@@ -779,9 +779,7 @@ def run_e2e(P, args, world):
     # Every rank reads the free memory before any rank pins, and all take the
     # most restrictive choice, so that they run the same collectives.
     barrier(world)
-    budget = _host_budget()
-    choice = 0 if budget is None or need_in + need_out <= budget else (1 if max(need_in, need_out) <= budget else 2)
-    choice = int(max_over_ranks(float(choice), world))
+    choice = int(max_over_ranks(float(host_buffer_choice(need_in, need_out, _host_budget())), world))
     if choice == 0:
         host_mode = "separate"
         host_in = {id(t): pinned(t) for t in inputs}
@@ -894,6 +892,14 @@ def run_e2e(P, args, world):
             "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h), "steps": steps,
             "ms_per_step": round(ms / steps, 3), "host_buffers": host_mode,
             "overlap": "host->device, compute and device->host on three streams, ordered by events per buffer"}
+
+
+def host_buffer_choice(need_in, need_out, budget):
+    """0: separate pinned input and output buffers; 1: one pool shared by
+    both; 2: no end-to-end figure.  budget None means unknown (assume room)."""
+    if budget is None or need_in + need_out <= budget:
+        return 0
+    return 1 if max(need_in, need_out) <= budget else 2
 
 
 def _host_budget():
