@@ -17,6 +17,18 @@
  *   lg_euler_step   same section: z_{k+1} = z_k + (sigma_{k+1} - sigma_k) v on
  *                   the schedule 0.909 -> 0.857 -> 0.667 -> 0.
  *
+ * and, from the same article's section "Where the 3.9x speedup comes from":
+ *
+ *   lg_mx_quantize, lg_lora_linear_mxfp8   the linear layer with its base term
+ *                   as MXFP8 GEMMs, activations re-quantized per call;
+ *   lg_lora_linear_swiglu_mxfp8   the MLP input projection with SwiGLU and
+ *                   the activation quantizer fused;
+ *   lg_lora_linear_euler   the step's last projection with the Euler update
+ *                   (and the bf16 copy of the new latent) fused;
+ *   lg_shift_ladder the sampler routes of "Open-H3-Regenerate-2K-IC"
+ *                   (wujieai.com) on HyperFlow's shift-12 table (host only);
+ *   lg_lora_linear_noalloc   lg_lora_linear without a caller workspace.
+ *
  * The pages name no random number generator.  This library draws eps from a
  * Philox4x32-10 stream (Salmon et al., "Parallel Random Numbers: As Easy as
  * 1, 2, 3", SC'11) with key = (seed mod 2^32, seed >> 32) and counter
