@@ -188,3 +188,17 @@ def test_host_validation_fused_and_mxfp8_entry_points():
     assert lg.lora_linear_euler_workspace_size(10, 100, 24, 64) == 0
     assert L.lg_mx_quantize(None, 4, 128, out, sc, None) == lg.LG_ERR_INVALID_ARG
     assert L.lg_mx_quantize(A16, 4, 96, out, sc, None) == lg.LG_ERR_UNSUPPORTED_SHAPE
+
+
+def test_mx_scale_bytes_host_arithmetic():
+    """One E8M0 byte per 32 values along K, rows padded to the 128-row groups
+    of the blocked layout (the layout the block-scaled MMAs read)."""
+    import lora_gemm_b200 as lg
+
+    assert lg.mx_scale_bytes(128, 128) == 128 * 4
+    assert lg.mx_scale_bytes(1, 128) == 128 * 4
+    assert lg.mx_scale_bytes(129, 256) == 256 * 8
+    assert lg.mx_scale_bytes(532800, 7168) == (532800 + 127) // 128 * 128 * 224
+    assert lg.mx_scale_bytes(0, 128) == 0
+    for bad in [(10, 96), (10, 64), (-1, 128), (10, 0)]:
+        assert lg.mx_scale_bytes(*bad) == 0
