@@ -43,3 +43,21 @@ def test_product_sources_do_not_mention_the_oracle_package():
         if name.endswith((".cu", ".cuh", ".h", ".inc")):
             text = open(os.path.join(csrc, name), encoding="utf-8").read()
             assert "oracle/" not in text and "import oracle" not in text, name
+
+
+def test_binding_fails_loudly_without_the_library(tmp_path):
+    """A copy of the package without liblora_gemm.so raises ImportError on
+    import: there is no CPU fallback to fall back to."""
+    import shutil
+    import subprocess
+    import sys
+
+    pkg = tmp_path / "lora_gemm_b200"
+    pkg.mkdir()
+    for name in ("__init__.py", "synth.py", "dist.py"):
+        shutil.copy(os.path.join(ROOT, "lora_gemm_b200", name), pkg / name)
+    code = ("import sys\nsys.path.insert(0, sys.argv[1])\n"
+            "try:\n    import lora_gemm_b200\nexcept ImportError as e:\n    print('ImportError', e)\n"
+            "else:\n    print('imported')\n")
+    out = subprocess.run([sys.executable, "-c", code, str(tmp_path)], capture_output=True, text=True, timeout=300)
+    assert out.stdout.startswith("ImportError"), out.stdout + out.stderr
