@@ -163,7 +163,7 @@ class Problem:
     """Device-resident inputs and outputs of one 2K step."""
 
     def __init__(self, w, dev, tokens=None, noise_offset=0):
-        from lora_gemm_b200 import synth
+        import synth
         import lora_gemm_b200 as lg
 
         self.w = w
@@ -468,7 +468,7 @@ def run_fusions(P, args, world, peaks):
     Fused and unfused calls alternate; each figure is a median.
     """
     import lora_gemm_b200 as lg
-    from lora_gemm_b200 import synth
+    import synth
 
     w, dev, R = P.w, P.up.device, P.R
     reps = max(args.steps, 5)
@@ -574,7 +574,7 @@ def bytes_per_kernel(P):
 
 def run_ours(args, rank, world, local):
     import lora_gemm_b200 as lg
-    from lora_gemm_b200 import synth
+    import synth
 
     peaks = load_peaks()
     dev = torch.device("cuda", torch.cuda.current_device())
@@ -934,7 +934,7 @@ class OracleStep:
     def __init__(self, w, tokens):
         import numpy as np
 
-        from lora_gemm_b200 import synth
+        import synth
 
         self.w = w
         self.tokens = tokens
@@ -992,10 +992,10 @@ def cpu_baseline(w, target_s=15.0):
 
 
 def run_reference(args, rank, world):
-    from lora_gemm_b200 import synth
+    import synth
 
     w = synth.WORKLOADS[args.workload]
-    per_step_s = 90.0 / max(1, args.steps + args.warmup)
+    per_step_s = getattr(args, "reference_seconds", 90.0) / max(1, args.steps + args.warmup)
     tokens = _oracle_tokens_for(w, per_step_s, 12288)
     step = OracleStep(w, tokens)
     for _ in range(args.warmup):
@@ -1044,6 +1044,8 @@ def main():
     ap.add_argument("--no-fusions", action="store_true", help="skip the fused-epilogue comparisons, the IC routes and the isolated elementwise runs")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    ap.add_argument("--reference-seconds", type=float, default=90.0,
+                    help="CPU seconds the oracle arm spends over all its warm-up and timed steps")
     ap.add_argument("--tokens", type=int, default=None,
                     help="override the token count of the linear layers (profiling runs only)")
     args = ap.parse_args()

@@ -4,7 +4,7 @@ Tolerances: Philox words bit-exact; eps within 2 FP32 ulp of the oracle's
 FP64 value rounded to FP32; re-noise and Euler within 2 ulp of the larger
 of the two blended terms (a result that cancels to near zero has no
 meaningful ulp of its own); the merge bit-exact (one FP32 rounding of s*A,
-an exact copy of B).  Inputs come from lora_gemm_b200.synth (torch
+an exact copy of B).  Inputs come from synth (torch
 generators), never from a kernel under test.
 """
 
@@ -13,7 +13,7 @@ import pytest
 import torch
 
 import lora_gemm_b200 as lg
-from lora_gemm_b200 import synth
+import synth
 from oracle import flow as oflow
 from oracle import lora as olora
 from oracle import noise as onoise

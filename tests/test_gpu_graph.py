@@ -13,7 +13,7 @@ import pytest
 import torch
 
 import lora_gemm_b200 as lg
-from lora_gemm_b200 import synth
+import synth
 
 pytestmark = pytest.mark.gpu
 DEV = "cuda"

@@ -14,7 +14,7 @@ import pytest
 import torch
 
 import lora_gemm_b200 as lg
-from lora_gemm_b200 import synth
+import synth
 from oracle import flow as oflow
 from oracle import noise as onoise
 from tests.util import ulp_diff, ulp_of

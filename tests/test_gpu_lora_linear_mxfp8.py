@@ -13,7 +13,7 @@ import pytest
 import torch
 
 import lora_gemm_b200 as lg
-from lora_gemm_b200 import synth
+import synth
 from oracle import lora as olora
 from oracle import mxfp8 as omx
 from tests.util import rel_fro

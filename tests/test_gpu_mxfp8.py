@@ -8,7 +8,7 @@ import pytest
 import torch
 
 import lora_gemm_b200 as lg
-from lora_gemm_b200 import synth
+import synth
 from oracle import mxfp8 as omx
 
 pytestmark = pytest.mark.gpu

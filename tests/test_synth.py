@@ -1,4 +1,4 @@
-"""The synthetic input recipe (lora_gemm_b200/synth.py) on the CPU: grid
+"""The synthetic input recipe (synth.py) on the CPU: grid
 shapes and token counts of the pages' workloads, per-tensor seeding (the same
 seed gives the same draw, different tensors and workloads differ) and the
 stated distributions -- x ~ N(0, 1) and W ~ N(0, 1/K) in bf16, A_i ~ N(0, 1/K)
@@ -9,7 +9,7 @@ import math
 import pytest
 import torch
 
-from lora_gemm_b200 import synth
+import synth
 
 CPU = "cpu"
 
