@@ -274,7 +274,9 @@ lg_status lg_lora_linear_euler(const void* x, const void* W, const float* A_cat,
  * loaded holds that memory until the process exits.  The call itself
  * allocates nothing (no cudaMalloc, cudaFree or allocating library routine).
  *
- *   - Result, validation, arithmetic and kernels are those of lg_lora_linear.
+ *   - Result, validation, arithmetic and kernels are those of lg_lora_linear;
+ *     its argument checks run first, so a bad argument gives the status
+ *     lg_lora_linear would give, before any CUDA call.
  *   - Limit: lg_lora_linear_workspace_size(M, K, N, R) must not exceed
  *     LG_NOALLOC_SCRATCH_BYTES (about 2 (K + N) R bytes; with R = 576 this is
  *     K + N <= 43,690, e.g. the 7168 -> 7168, 7168 -> 21504 and
@@ -282,7 +284,11 @@ lg_status lg_lora_linear_euler(const void* x, const void* W, const float* A_cat,
  *     launches nothing.
  *   - The first call on a device looks up the array's device address on that
  *     device (cudaGetSymbolAddress, with that device current); make that
- *     first call before any stream capture.
+ *     first call before any stream capture.  The address belongs to the
+ *     current CUDA context: it is cached per device and context, so the first
+ *     call after a context was destroyed and recreated (cudaDeviceReset), or
+ *     under another context, looks it up again (and is then also a first
+ *     call in the sense above).
  *   - Every call uses the same array.  Calls that can overlap on the GPU
  *     (different streams without ordering between them) race on it; keep
  *     such calls on one stream or order them with events.

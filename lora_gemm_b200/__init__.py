@@ -26,6 +26,10 @@ LG_ERR_CUDA = 5
 LG_ERR_DEVICE_TIMEOUT = 6
 LG_ERR_NOT_SM100 = 7
 
+# Size of the built-in scratch array of lg_lora_linear_noalloc (the header's
+# LG_NOALLOC_SCRATCH_BYTES).
+LG_NOALLOC_SCRATCH_BYTES = 48 << 20
+
 # Exported C symbols and their ctypes signatures (the header's declarations).
 _c_void_p = ctypes.c_void_p
 _SIGNATURES = {

@@ -4,6 +4,8 @@
 #include <cmath>
 #include <mutex>
 
+#include <cudaTypedefs.h>
+
 #include "../../include/lora_gemm.h"
 #include "lg_internal.h"
 
@@ -223,9 +225,12 @@ struct EulerOut {
   float dt;
 };
 
+// check_only: validate everything but the workspace (the caller brings its
+// own, distinct from every argument) and the device, launch nothing.
 lg_status lora_linear_impl(const void* x, const void* W, const float* A_cat, const float* B_cat, void* y, int64_t M,
                            int K, int N, int R, void* workspace, size_t ws_bytes, void* stream,
-                           const MxOperands* mx, const SwigluOut* sw = nullptr, const EulerOut* eu = nullptr) {
+                           const MxOperands* mx, const SwigluOut* sw = nullptr, const EulerOut* eu = nullptr,
+                           bool check_only = false) {
   if (M < 0 || K < 0 || N < 0 || R < 0) return LG_ERR_INVALID_ARG;
   // The Euler output takes any N >= 1 (its epilogue writes single values).
   const bool n_ok = eu ? N >= 1 : (N >= 32 && N % 32 == 0);
@@ -250,8 +255,8 @@ lg_status lora_linear_impl(const void* x, const void* W, const float* A_cat, con
   if (mx && (!aligned16(mx->xq) || !aligned16(mx->xsf) || !aligned16(mx->wq) || !aligned16(mx->wsf)))
     return LG_ERR_MISALIGNED;
   if (R > 0 && (!aligned16(A_cat) || !aligned16(B_cat))) return LG_ERR_MISALIGNED;
-  const size_t need = R > 0 ? factor_copy_bytes(K, N, R) : 0;
-  if (R > 0) {
+  const size_t need = R > 0 && !check_only ? factor_copy_bytes(K, N, R) : 0;
+  if (R > 0 && !check_only) {
     if (!workspace || ws_bytes < need) return LG_ERR_WORKSPACE;
     if (!aligned16(workspace)) return LG_ERR_MISALIGNED;
   }
@@ -290,7 +295,7 @@ lg_status lora_linear_impl(const void* x, const void* W, const float* A_cat, con
   if (M == 0) return LG_OK;
   int sms = 0;
   lg_status st = current_device(&sms);
-  if (st != LG_OK) return st;
+  if (st != LG_OK || check_only) return st;
   cudaStream_t s = as_stream(stream);
   uint16_t* wsA = nullptr;
   uint16_t* wsB = nullptr;
@@ -339,6 +344,42 @@ lg_status lora_linear_impl(const void* x, const void* W, const float* A_cat, con
 }
 
 }  // namespace
+
+}  // extern "C"
+
+namespace lg {
+
+int check_lora_linear(const void* x, const void* W, const float* A_cat, const float* B_cat, const void* y,
+                      int64_t M, int K, int N, int R) {
+  return lora_linear_impl(x, W, A_cat, B_cat, const_cast<void*>(y), M, K, N, R, nullptr, 0, nullptr, nullptr,
+                          nullptr, nullptr, true);
+}
+
+bool current_context_id(unsigned long long* id) {
+  static PFN_cuCtxGetCurrent_v4000 get_current = nullptr;
+  static PFN_cuCtxGetId_v12000 get_id = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_current = reinterpret_cast<PFN_cuCtxGetCurrent_v4000>(p);
+    p = nullptr;
+    if (cudaGetDriverEntryPoint("cuCtxGetId", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_id = reinterpret_cast<PFN_cuCtxGetId_v12000>(p);
+    cudaGetLastError();
+  });
+  if (!get_current || !get_id) return false;
+  CUcontext ctx = nullptr;
+  if (get_current(&ctx) != CUDA_SUCCESS || ctx == nullptr) return false;
+  return get_id(ctx, id) == CUDA_SUCCESS;
+}
+
+}  // namespace lg
+
+extern "C" {
 
 lg_status lg_lora_linear(const void* x, const void* W, const float* A_cat, const float* B_cat, void* y, int64_t M,
                          int K, int N, int R, void* workspace, size_t ws_bytes, void* stream) {

@@ -89,4 +89,17 @@ void set_variant_override(int v);
 // Device error word of the current device: read and clear (synchronous on s).
 cudaError_t read_and_clear_device_error(cudaStream_t s, int* value);
 
+// The driver's process-unique id of the calling thread's current CUDA
+// context.  False when no context is current or the driver cannot say; a
+// per-device cache keyed on this id notices a context that was destroyed
+// and recreated (cudaDeviceReset) or a different context made current.
+bool current_context_id(unsigned long long* id);
+
+// Every check lg_lora_linear makes on its arguments except those on the
+// workspace, then (for M > 0) the current device's compute capability, in
+// the same order and with the same status codes; launches nothing.  Returns
+// an lg_status value.
+int check_lora_linear(const void* x, const void* W, const float* A_cat, const float* B_cat, const void* y,
+                      int64_t M, int K, int N, int R);
+
 }  // namespace lg

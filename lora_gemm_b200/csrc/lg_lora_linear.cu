@@ -1198,11 +1198,17 @@ int max_active_clusters(const void* kernel, int variant, int dev, int cluster, s
   return n;
 }
 
+// Function attributes belong to the context the kernels are loaded in: the
+// cache is keyed on the device and the current context's id (without an id
+// the attributes are set on every launch).
 cudaError_t configure_kernels(int dev) {
   static std::mutex mu;
   static bool configured[64] = {};
+  static unsigned long long context[64] = {};
   std::lock_guard<std::mutex> lock(mu);
-  if (dev >= 0 && dev < 64 && configured[dev]) return cudaSuccess;
+  unsigned long long ctx = 0;
+  const bool have_ctx = current_context_id(&ctx);
+  if (dev >= 0 && dev < 64 && have_ctx && configured[dev] && context[dev] == ctx) return cudaSuccess;
   const void* kernels[3] = {(const void*)k_lora_linear<false, false>, (const void*)k_lora_linear<true, false>,
                             (const void*)k_lora_linear<true, true>};
   for (const void* k : kernels) {
@@ -1210,7 +1216,10 @@ cudaError_t configure_kernels(int dev) {
     if (e == cudaSuccess) e = cudaFuncSetAttribute(k, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
     if (e != cudaSuccess) return e;
   }
-  if (dev >= 0 && dev < 64) configured[dev] = true;
+  if (dev >= 0 && dev < 64) {
+    configured[dev] = have_ctx;
+    context[dev] = ctx;
+  }
   return cudaSuccess;
 }
 

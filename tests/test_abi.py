@@ -202,3 +202,38 @@ def test_mx_scale_bytes_host_arithmetic():
     assert lg.mx_scale_bytes(0, 128) == 0
     for bad in [(10, 96), (10, 64), (-1, 128), (10, 0)]:
         assert lg.mx_scale_bytes(*bad) == 0
+
+
+def test_noalloc_reports_the_same_status_as_lg_lora_linear():
+    """lg_lora_linear_noalloc runs lg_lora_linear's argument checks before its
+    own scratch limit and before any CUDA call, so a bad argument gives the
+    same status from both entry points (CPU: nothing here reaches a device)."""
+    import ctypes
+
+    import lora_gemm_b200 as lg
+
+    L = lg.lib
+    base = 0x7F0000000000
+    x, W, A, B, y, ws = (ctypes.c_void_p(base + i * (1 << 36)) for i in range(6))
+    ws_bytes = 1 << 30
+    cases = {
+        "null x": ((None, W, A, B, y, 256, 1024, 1024, 576), lg.LG_ERR_INVALID_ARG),
+        "null y": ((x, W, A, B, None, 256, 1024, 1024, 576), lg.LG_ERR_INVALID_ARG),
+        "null A_cat": ((x, W, None, B, y, 256, 1024, 1024, 576), lg.LG_ERR_INVALID_ARG),
+        "misaligned x": ((ctypes.c_void_p(base + 8), W, A, B, y, 256, 1024, 1024, 576), lg.LG_ERR_MISALIGNED),
+        "K not a multiple of 64": ((x, W, A, B, y, 256, 1000, 1024, 576), lg.LG_ERR_UNSUPPORTED_SHAPE),
+        "rank not a multiple of 64": ((x, W, A, B, y, 256, 1024, 1024, 96), lg.LG_ERR_UNSUPPORTED_SHAPE),
+        "y overlaps x": ((x, W, A, B, ctypes.c_void_p(base + 1024), 256, 1024, 1024, 576), lg.LG_ERR_INVALID_ARG),
+        "negative M": ((x, W, A, B, y, -1, 1024, 1024, 576), lg.LG_ERR_INVALID_ARG),
+    }
+    for name, (args, want) in cases.items():
+        a = args[:9]
+        got_ws = L.lg_lora_linear(*a, ws, ws_bytes, None)
+        got_na = L.lg_lora_linear_noalloc(*a, None)
+        assert got_ws == got_na == want, f"{name}: lg_lora_linear {got_ws}, noalloc {got_na}, want {want}"
+    # An empty batch with a valid shape launches nothing and needs no device.
+    assert L.lg_lora_linear_noalloc(x, W, A, B, y, 0, 1024, 1024, 576, None) == lg.LG_OK
+    # Valid arguments but a shape beyond the built-in scratch: refused as a too-small workspace would be.
+    assert L.lg_lora_linear_noalloc(x, W, A, B, y, 0, 32768, 32768, 576, None) == lg.LG_ERR_WORKSPACE
+    assert L.lg_lora_linear(x, W, A, B, y, 0, 32768, 32768, 576, ws, lg.LG_NOALLOC_SCRATCH_BYTES, None) == \
+        lg.LG_ERR_WORKSPACE

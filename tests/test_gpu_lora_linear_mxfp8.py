@@ -104,6 +104,36 @@ def test_full_size_sampled_rows(name, layer):
     assert rel_fro(y_rows, ref) <= TOL
 
 
+def test_full_size_d_to_3d_sampled_rows_and_tiles():
+    """The 2K grid's d -> 3d layer (7168 -> 21504, the widest N the step
+    runs): 258 sampled tokens (first and last included) times 12 of the 84
+    output tiles of 256 columns (first and last included); output columns
+    depend only on their own W rows, so the oracle takes those rows alone."""
+    w = synth.WORKLOADS["2k"]
+    layer = 1
+    K, N = w.shapes[layer]
+    x = synth.activations(w, K, layer, DEV)
+    W = synth.weight(w, layer, DEV)
+    As, Bs = synth.adapters(w, layer, DEV)
+    A_cat, B_cat = lg.lora_merge(As, Bs, synth.ADAPTER_SCALES)
+    y = lg.lora_linear_mxfp8(x, lg.mx_quantize(x), lg.mx_quantize(W), A_cat, B_cat)
+    assert lg.get_last_device_error() == lg.LG_OK
+    rng = np.random.default_rng(w.seed * 10 + layer + 1)
+    rows = np.unique(np.concatenate([rng.choice(w.tokens, 256, replace=False), [0, w.tokens - 1]]))
+    tiles = np.unique(np.concatenate([rng.choice(N // 256, 10, replace=False), [0, N // 256 - 1]]))
+    cols = (tiles[:, None] * 256 + np.arange(256)[None, :]).reshape(-1)
+    ridx = torch.as_tensor(rows, device=DEV)
+    cidx = torch.as_tensor(cols, device=DEV)
+    y_s = _np64(y.index_select(0, ridx).index_select(1, cidx))
+    x_rows = _np64(x.index_select(0, ridx))
+    W_s = _np64(W.index_select(0, cidx))
+    B_s = _np64(B_cat.index_select(0, cidx))
+    del x, y
+    torch.cuda.empty_cache()
+    ref = omx.lora_linear_mxfp8(x_rows, W_s, _np64(A_cat), B_s)
+    assert rel_fro(y_s, ref) <= TOL
+
+
 def test_wait_timeout_is_reported():
     x, W, A, B = _layer(2048, 1024, 1792, 576, seed=19)
     lg.set_wait_limit_ns(1)

@@ -20,6 +20,7 @@ import pytest
 import torch
 
 import lora_gemm_b200 as lg
+import synth
 from oracle import mxfp8 as omx
 from tests.util import rel_fro
 
@@ -124,3 +125,48 @@ def test_swiglu_wait_timeout_is_reported():
     codes, scales = lg.lora_linear_swiglu_mxfp8(x, xq, wq, A, B)
     assert lg.get_last_device_error() == lg.LG_OK
     _check(x, W2, A, B, R, codes, scales)
+
+
+def test_swiglu_at_the_benched_shape_sampled():
+    """The shape the step's fused MLP input projection is timed on: a quarter
+    of the 2K grid (133,120 tokens), d = 7168 -> 2 x 28,672, merged rank 576,
+    drawn as for the timing.  258 sampled tokens (first and last included)
+    times 16 of the 224 output tiles of 128 columns (first and last
+    included); a tile's outputs depend only on its gate rows and up rows of
+    W2 and B_cat, so the oracle takes those rows alone (blocks of 32 along
+    the outputs stay whole)."""
+    w = synth.WORKLOADS["2k"]
+    K, N2 = synth.mlp_in_shape(w)
+    F = N2 // 2
+    M = (w.tokens // 4) // 128 * 128
+    x = synth.activations(w, K, 0, DEV, M=M)
+    W2 = synth.weight(w, synth.MLP_IN_LAYER, DEV, shape=(K, N2))
+    As, Bs = synth.adapters(w, synth.MLP_IN_LAYER, DEV, shape=(K, N2))
+    A_cat, B_cat = lg.lora_merge(As, Bs, synth.ADAPTER_SCALES)
+    del As, Bs
+    codes, scales = lg.lora_linear_swiglu_mxfp8(x, lg.mx_quantize(x), lg.mx_quantize(W2), A_cat, B_cat)
+    assert lg.get_last_device_error() == lg.LG_OK
+    rng = np.random.default_rng(17)
+    rows = np.unique(np.concatenate([rng.choice(M, 256, replace=False), [0, M - 1]]))
+    tiles = np.unique(np.concatenate([rng.choice(F // 128, 14, replace=False), [0, F // 128 - 1]]))
+    cols = (tiles[:, None] * 128 + np.arange(128)[None, :]).reshape(-1)
+    w_rows = np.concatenate([cols, F + cols])
+    ridx = torch.as_tensor(rows, device=DEV)
+    got_codes = codes.index_select(0, ridx).index_select(1, torch.as_tensor(cols, device=DEV)).cpu().numpy()
+    blocks = (tiles[:, None] * 4 + np.arange(4)[None, :]).reshape(-1)
+    r = rows[:, None]
+    kb = blocks[None, :]
+    off = ((r // 128) * (F // 128) + kb // 4) * 512 + 16 * (r % 128 % 32) + 4 * (r % 128 // 32) + kb % 4
+    got_exps = scales.cpu().numpy()[off].astype(np.int32) - 127
+    x_rows = _np64(x.index_select(0, ridx))
+    widx = torch.as_tensor(w_rows, device=DEV)
+    W2_s = _np64(W2.index_select(0, widx))
+    B_s = _np64(B_cat.index_select(0, widx))
+    del x, W2, codes, scales
+    torch.cuda.empty_cache()
+    s, (ref_codes, ref_exps) = omx.swiglu_mxfp8(x_rows, W2_s, _np64(A_cat), B_s)
+    got = omx.mx_dequantize(got_codes, got_exps)
+    ref = omx.mx_dequantize(ref_codes, ref_exps)
+    assert rel_fro(got, ref) <= (1e-2 * 2.0 ** -4) ** 0.5
+    assert rel_fro(got, s) <= 2.0 ** -4
+    assert np.mean(got_exps == ref_exps) >= 0.99
