@@ -470,6 +470,48 @@ def _time_alternating(f, g, reps, world):
     return max_over_ranks(statistics.median(tf), world), max_over_ranks(statistics.median(tg), world)
 
 
+def run_library_ab(P, args, world, peaks):
+    """Each layer of the step against the unfused library composition of the
+    same arithmetic, timed alternately (medians, CUDA events on the current
+    stream): cuBLAS bf16 y = x W^T, cuBLAS h = x A_cat^T written to HBM
+    (bf16, [M, R]), cuBLAS y += h B_cat^T, with the factors' bf16 copies made
+    by torch inside the timed call (the fused call makes its own inside too).
+    Context for the fusion: the fused kernel saves the h round trip (2 M R
+    bytes each way) and the separate passes."""
+    import lora_gemm_b200 as lg
+
+    out = []
+    h = torch.empty((P.M, P.R), dtype=torch.bfloat16, device=P.up.device)
+    reps = 3
+    for k, L in enumerate(P.layers):
+        x, W, A, B, y, ws = L["x"], L["W"], L["A_cat"], L["B_cat"], L["y"], L["ws"]
+
+        def fused():
+            lg.lora_linear(x, W, A, B, y=y, workspace=ws)
+
+        def unfused():
+            A16 = A.to(torch.bfloat16)
+            B16 = B.to(torch.bfloat16)
+            torch.matmul(x, W.t(), out=y)
+            torch.matmul(x, A16.t(), out=h)
+            y.addmm_(h, B16.t())
+
+        f_ms, u_ms = _time_alternating(fused, unfused, reps, world)
+        fl = layer_flops(P.M, L["K"], L["N"], P.R)
+        out.append({"k_n": [L["K"], L["N"]], "fused_ms": round(f_ms, 3), "unfused_cublas_ms": round(u_ms, 3),
+                    "fused_tflops": round(fl / (f_ms * 1e-3) / 1e12, 1),
+                    "unfused_tflops": round(fl / (u_ms * 1e-3) / 1e12, 1),
+                    "fused_speedup": round(u_ms / f_ms, 3)})
+    del h
+    torch.cuda.empty_cache()
+    status = lg.get_last_device_error()
+    if status != lg.LG_OK:
+        raise SystemExit(f"device error during the library A/B: {lg.status_string(status)}")
+    return {"per_layer": out, "reps": reps,
+            "note": "fused lg_lora_linear against cuBLAS x W^T + cuBLAS h = x A^T (h in HBM) + cuBLAS y += h B^T, "
+                    "calls alternating, medians; algorithmic FLOPs 2 M (K N + K R + R N) for both"}
+
+
 def run_fusions(P, args, world, peaks):
     """Epilogue fusions beside the step, each against its unfused form:
 
@@ -750,6 +792,7 @@ def run_ours(args, rank, world, local):
     if not args.no_mxfp8:
         result["mxfp8"] = run_mxfp8(P, args, world, peaks)
     if not args.no_fusions:
+        result["library_ab"] = run_library_ab(P, args, world, peaks)
         result["fusions"] = run_fusions(P, args, world, peaks)
         result["ic_routes"] = run_ic_routes(P, args, world, peaks)
         result["elementwise_isolated"] = run_elementwise_isolated(P, args, world, peaks)
@@ -782,12 +825,21 @@ def run_workloads(names, args, world, rank, dev, peaks):
         w = synth.WORKLOADS[name]
         P = Problem(w, dev, noise_offset=_dist().noise_offset(rank, w.latent_numel), lean=True)
         torch.cuda.synchronize()
-        ms, per, launches, clk = time_steps(P, args, world, rank, dev)
+        # Enough timed steps for >= 1.5 s under the clock sampler (200 ms period).
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        run_step(P)
+        e1.record()
+        torch.cuda.synchronize()
+        one_ms = max_over_ranks(e0.elapsed_time(e1), world)
+        wargs = argparse.Namespace(**vars(args))
+        wargs.steps = max(args.steps, min(2000, int(1500.0 / max(one_ms, 1e-3)) + 1))
+        ms, per, launches, clk = time_steps(P, wargs, world, rank, dev)
         kernels, flops, tflops = kernel_report(P, per, peaks)
         rec = {
             "latent": list(w.latent_shape), "tokens": P.M, "d": w.d, "layers_k_n": [list(x) for x in w.shapes],
-            "tokens_per_s": round(_dist().whole_job_rate(P.M, world, args.steps, ms), 1),
-            "ms_per_step": round(ms / args.steps, 3), "steps": args.steps, "warmup": args.warmup,
+            "tokens_per_s": round(_dist().whole_job_rate(P.M, world, wargs.steps, ms), 1),
+            "ms_per_step": round(ms / wargs.steps, 3), "steps": wargs.steps, "warmup": args.warmup,
             "kernels": kernels, "clocks": clk, "gpu_launches": int(launches),
             "inputs": "lean: layer activations are views of one buffer of the widest K, outputs share one buffer",
         }

@@ -54,84 +54,96 @@ __device__ __forceinline__ Words4 philox4x32_10(uint64_t block, uint32_t k0, uin
 // ---------------------------------------------------------------------------
 struct BmLogEntry {
   double inv_c;  // 1 / c_i cut to 28 significant bits, c_i = 1 + i / 256
-  double L;      // -ln(inv_c), or -ln(2 inv_c) for i > LG_BM_LOG_SWITCH
+  double y;      // -2 times the log term: 2 ln(inv_c), or 2 ln(2 inv_c) for i > LG_BM_LOG_SWITCH
 };
 struct BmTrigEntry {
-  double s, c;  // sin, cos of 2 pi i / 256 (exact 0 and +-1 at quarter turns)
+  double s, c;  // sin, cos of 2 pi i / 1024 (exact 0 and +-1 at quarter turns)
 };
 struct BmTables {
   const BmLogEntry* log;   // 257 entries
-  const BmTrigEntry* trig; // 256 entries
+  const BmTrigEntry* trig; // 1024 entries
 };
 constexpr int kBmLogSwitch = 106;
+constexpr int kBmTrigBits = 10;  // 1024 trig entries
 
 __device__ __forceinline__ double bits_to_double(uint64_t b) { return __longlong_as_double((long long)b); }
+__device__ __forceinline__ double hilo_to_double(uint32_t hi, uint32_t lo) {
+  return __hiloint2double((int)hi, (int)lo);
+}
 
-// ln(n 2^-24) for an integer n in [1, 2^24] (Tang's table method).  With
-// n = m 2^kf, m in [1, 2), the nearest grid point c_i = 1 + i/256 gives
+// y = -2 ln(n 2^-24) for an integer n in [1, 2^24] (Tang's table method).
+// With n = m 2^kf, m in [1, 2), the nearest grid point c_i = 1 + i/256 gives
 // r = m inv_c - 1 exactly (m has <= 24 significant bits, inv_c 28) and
-// |r| <= 2^-9 + 2^-27, so log1p(r) to the r^6 term is within 2^-56 |r|.
-// Past c = sqrt 2 the entry already holds ln(c/2) and the exponent is one
-// higher, so a nonzero multiple of ln 2 always dominates the table term
-// (|ln u1| >= ln 2 - 0.35) and no step cancels.
-__device__ __forceinline__ double ln_grid24(uint32_t n, const BmLogEntry* tab) {
-  const int kf = 31 - __clz(n);
-  const uint32_t top = n << (31 - kf);                      // leading one at bit 31
-  const int i = (int)(((top >> 22) + 1u) >> 1) - 256;       // 0..256
+// |r| <= 2^-9 + 2^-27, so -2 log1p(r) = -2 r + r^2 q(r), q to the r^4 term
+// (the r^6 term of log1p), is within 2^-56 |r|.  Past c = sqrt 2 the entry
+// already holds the term of c/2 and the exponent is one higher, so a nonzero
+// multiple of ln 2 always dominates the table term (|ln u1| >= ln 2 - 0.35)
+// and no step cancels by more than a factor of two.
+__device__ __forceinline__ double neg2_ln_grid24(uint32_t n, const BmLogEntry* tab) {
+  const uint32_t lz = __clz(n);                             // 7..31 (kf = 31 - lz)
+  const uint32_t top = n << lz;                             // leading one at bit 31
+  const uint32_t i = (((top >> 22) + 1u) >> 1) - 256u;      // 0..256
   const BmLogEntry e = tab[i];
-  const int j = 24 - kf - (i > kBmLogSwitch ? 1 : 0);        // 0..24
-  // m = n 2^-kf assembled from the bits of n (exact)
-  const double m = bits_to_double(((uint64_t)n << (52 - kf)) + ((uint64_t)1022 << 52));
+  const uint32_t j = lz - 7u - (i > (uint32_t)kBmLogSwitch ? 1u : 0u);  // 24 - kf (- 1): 0..24
+  // m = n 2^-kf in [1, 2) from the bits of top (exact)
+  const double m = hilo_to_double(0x3FF00000u | ((top >> 11) & 0xFFFFFu), top << 21);
   const double r = fma(m, e.inv_c, -1.0);
-  double p = -1.0 / 6.0;
-  p = fma(p, r, 1.0 / 5.0);
-  p = fma(p, r, -1.0 / 4.0);
-  p = fma(p, r, 1.0 / 3.0);
-  p = fma(p, r, -0.5);
-  const double log1p_r = fma(r * r, p, r);
+  double q = 1.0 / 3.0;
+  q = fma(q, r, -2.0 / 5.0);
+  q = fma(q, r, 1.0 / 2.0);
+  q = fma(q, r, -2.0 / 3.0);
+  q = fma(q, r, 1.0);
   // (double)j from the bits of 2^52 + j
-  const double jd = bits_to_double(0x4330000000000000ull + (uint64_t)j) - 0x1p52;
-  return fma(-jd, 0.6931471805599453094, e.L + log1p_r);
+  const double jd = hilo_to_double(0x43300000u, j) - 0x1p52;
+  const double base = fma(jd, 1.3862943611198906188, e.y);  // 2 j ln 2 + table term
+  return fma(r * r, q, fma(-2.0, r, base));
 }
 
 // sqrt(y) for y = +-0 or y in [2^-24, 64): an FP32 reciprocal square root
 // seed, one Newton step on 1/sqrt(y) in double (relative error ~2^-44), then
 // one correction of y / sqrt(y) (error ~2^-88 before the final rounding).
 __device__ __forceinline__ double sqrt_seeded(double y) {
-  const uint32_t hi = max((uint32_t)__double2hiint(y) & 0x7FFFFFFFu, 0x3E700000u);  // finite seed at y = +-0
+  // max as signed: -0 (high word 0x80000000) takes the finite seed too
+  const uint32_t hi = (uint32_t)max(__double2hiint(y), 0x3E700000);
   const float yf = __uint_as_float((hi - (896u << 20)) << 3);        // y truncated to FP32
   float rf;
   asm("rsqrt.approx.ftz.f32 %0, %1;" : "=f"(rf) : "f"(yf));
-  double r = bits_to_double(((uint64_t)__float_as_uint(rf) << 29) + ((uint64_t)896 << 52));
+  const uint32_t rb = __float_as_uint(rf);
+  double r = hilo_to_double((rb >> 3) + (896u << 20), rb << 29);
   const double t = y * r;
-  r = fma(0.5 * r, fma(-t, r, 1.0), r);
+  const double hr = 0.5 * r;
+  r = fma(hr, fma(-t, r, 1.0), r);
   const double s0 = y * r;
   return fma(fma(-s0, s0, y), 0.5 * r, s0);
 }
 
 // sin and cos of 2 pi b 2^-24 for an integer b in [0, 2^24): the nearest
-// 1/256 turn comes from the table, the remainder theta (|theta| <= pi/256,
-// exact integer times 2 pi 2^-24) from short Maclaurin series (truncation
-// below 1e-20 relative), combined by the angle-addition formulas.  Near a
-// zero of sin or cos the table term is exactly zero, so the result keeps full
-// relative accuracy.
+// 1/1024 turn comes from the table, the remainder theta (|theta| <= pi/1024,
+// an exact integer rd times K = 2 pi 2^-24) from short Maclaurin series
+// (sin to theta^5, cos - 1 to theta^4: truncation below 2e-19 relative),
+// combined by the angle-addition formulas.  Near a zero of sin or cos the
+// table term is exactly zero, so the result keeps full relative accuracy.
 __device__ __forceinline__ void sincos_turn24(uint32_t b, const BmTrigEntry* tab, double& s, double& c) {
-  const uint32_t iu = ((b >> 15) + 1u) >> 1;                 // nearest multiple of 2^16, 0..256
-  const int32_t ri = (int32_t)b - (int32_t)(iu << 16);       // -2^15 .. 2^15 - 1
-  const BmTrigEntry t = tab[iu & 255u];
-  // (double)ri from the bits of 1.5 2^52 + ri
-  const double rd = bits_to_double(0x4338000000000000ull + (uint64_t)(int64_t)ri) - 0x1.8p52;
-  const double th = rd * (6.283185307179586 * 0x1p-24);
-  const double z = th * th;
-  const double sth = fma(th * z, fma(z, fma(z, -1.0 / 5040.0, 1.0 / 120.0), -1.0 / 6.0), th);
-  const double cm1 = z * fma(z, fma(z, -1.0 / 720.0, 1.0 / 24.0), -0.5);  // cos(theta) - 1
+  constexpr int kShift = 24 - kBmTrigBits;                   // 14
+  const uint32_t iu = ((b >> (kShift - 1)) + 1u) >> 1;       // nearest table point, 0..1024
+  // rd = b - iu 2^14 in [-2^13, 2^13), as a double from the bits of
+  // 2^52 + (rd + 2^13)
+  const uint32_t ri = b - (iu << kShift) + (1u << (kShift - 1));
+  const BmTrigEntry t = tab[iu & ((1u << kBmTrigBits) - 1u)];
+  const double rd = hilo_to_double(0x43300000u, ri) - (0x1p52 + 0x1p13);
+  constexpr double K = 6.283185307179586476925 * 0x1p-24;
+  constexpr double S3 = -K * K * K / 6.0, S5 = K * K * K * K * K / 120.0;
+  constexpr double C2 = -K * K / 2.0, C4 = K * K * K * K / 24.0;
+  const double z = rd * rd;                                  // exact (|rd| <= 2^13)
+  const double sth = rd * fma(z, fma(z, S5, S3), K);         // sin(theta)
+  const double cm1 = z * fma(z, C4, C2);                     // cos(theta) - 1
   s = fma(t.s, cm1, fma(t.c, sth, t.s));
   c = fma(t.c, cm1, fma(-t.s, sth, t.c));
 }
 
 __device__ __forceinline__ void box_muller(uint32_t a, uint32_t b, const BmTables& tab, double& e_cos,
                                            double& e_sin) {
-  const double rho = sqrt_seeded(-2.0 * ln_grid24((a >> 8) + 1u, tab.log));
+  const double rho = sqrt_seeded(neg2_ln_grid24((a >> 8) + 1u, tab.log));
   double s, c;
   sincos_turn24(b >> 8, tab.trig, s, c);
   e_cos = rho * c;

@@ -19,9 +19,14 @@ namespace lg {
 namespace {
 
 constexpr int kThreads = 256;
-// The FP64 Box-Muller kernels are issue-bound: 4 blocks per SM (64 registers
-// a thread) beat 8 blocks (32 registers) by 3 % on the 2K latent.
-constexpr int kBmBlocksPerSm = 4;
+// The FP64 Box-Muller kernels are issue-bound.  On the 2K latent, with each
+// thread working on three Philox blocks at once (kBmUnroll), 2 blocks per SM
+// (122 registers a thread) gave 2.93 TB/s for the re-noise; one block at a
+// time gave 2.60 at 4 blocks per SM, two at a time 2.67-2.77 at 2-4.
+#ifndef LG_BM_BLOCKS_PER_SM
+#define LG_BM_BLOCKS_PER_SM 2
+#endif
+constexpr int kBmBlocksPerSm = LG_BM_BLOCKS_PER_SM;
 
 static_assert(LG_BM_LOG_SWITCH == kBmLogSwitch, "log table built for another switch point");
 __device__ const BmLogEntry g_bm_log[LG_BM_LOG_ENTRIES] = LG_BM_LOG_TABLE;
@@ -55,50 +60,91 @@ __device__ __forceinline__ void normals4(uint64_t block, uint32_t k0, uint32_t k
   box_muller(r.w2, r.w3, tab, e[2], e[3]);
 }
 
-__global__ void __launch_bounds__(kThreads, kBmBlocksPerSm) k_philox_normal(float* __restrict__ eps, int64_t n, uint32_t k0,
-                                                            uint32_t k1, uint64_t block0) {
-  __shared__ BmLogEntry s_log[LG_BM_LOG_ENTRIES];
-  __shared__ BmTrigEntry s_trig[LG_BM_TRIG_ENTRIES];
-  const BmTables tab = stage_bm_tables(s_log, s_trig);
-  const int64_t n_blocks = (n + 3) / 4;
-  for (int64_t b = gtid(); b < n_blocks; b += gstride()) {
+// The normal stream (RENOISE = false: eps = the FP32 roundings) or the
+// re-noise x = (1 - sigma) up + sigma eps (blended in double from the
+// unrounded eps and rounded once to FP32) over the elements [0, 4 nb + tail)
+// of one launch, whose element 0 is global element 4 block0.  Threads stride
+// over the nb full Philox blocks (one float4 each) with 32-bit indices; each
+// loads its next block of up before the FP64 work on the current one, so the
+// load's DRAM latency hides behind that work; the `tail` < 4 elements past
+// them go to thread 0 of block 0.  x may alias up (each element is read
+// before it is written by the same thread), so neither pointer is restrict.
+#ifndef LG_BM_UNROLL
+#define LG_BM_UNROLL 3
+#endif
+constexpr int kBmUnroll = LG_BM_UNROLL;  // Philox blocks a thread works on at once
+
+template <bool RENOISE>
+__device__ __forceinline__ void normal_stream(const float* up, float* out, uint32_t nb, uint32_t tail, double sigma,
+                                              uint32_t k0, uint32_t k1, uint64_t block0, const BmTables& tab) {
+  const double keep = 1.0 - sigma;
+  const uint32_t stride = gridDim.x * blockDim.x;
+  const uint32_t first = blockIdx.x * blockDim.x + threadIdx.x;
+  const float4* up4 = reinterpret_cast<const float4*>(up);
+  float4* out4 = reinterpret_cast<float4*>(out);
+  constexpr int U = kBmUnroll;
+  float4 u_next[U];
+#pragma unroll
+  for (int k = 0; k < U; ++k) {
+    u_next[k] = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (RENOISE && first + k * stride < nb) u_next[k] = __ldcs(up4 + first + k * stride);
+  }
+  for (uint32_t b = first; b < nb; b += U * stride) {
+    float4 u[U];
+#pragma unroll
+    for (int k = 0; k < U; ++k) {
+      u[k] = u_next[k];
+      const uint32_t bn = b + (U + k) * stride;
+      if (RENOISE && bn < nb) u_next[k] = __ldcs(up4 + bn);
+    }
+    // The U blocks are independent: their FP64 chains interleave.  A block
+    // past nb is computed but not stored.
+    double e[U][4];
+#pragma unroll
+    for (int k = 0; k < U; ++k) normals4(block0 + b + k * stride, k0, k1, tab, e[k]);
+#pragma unroll
+    for (int k = 0; k < U; ++k) {
+      if (k > 0 && b + k * stride >= nb) break;
+      float4 o;
+      if constexpr (RENOISE) {
+        o.x = (float)fma(sigma, e[k][0], keep * (double)u[k].x);
+        o.y = (float)fma(sigma, e[k][1], keep * (double)u[k].y);
+        o.z = (float)fma(sigma, e[k][2], keep * (double)u[k].z);
+        o.w = (float)fma(sigma, e[k][3], keep * (double)u[k].w);
+      } else {
+        o = make_float4((float)e[k][0], (float)e[k][1], (float)e[k][2], (float)e[k][3]);
+      }
+      __stcs(out4 + b + k * stride, o);
+    }
+  }
+  if (tail && first == 0) {
     double e[4];
-    normals4(block0 + (uint64_t)b, k0, k1, tab, e);
-    if (4 * b + 4 <= n) {
-      reinterpret_cast<float4*>(eps)[b] = make_float4((float)e[0], (float)e[1], (float)e[2], (float)e[3]);
-    } else {
-      for (int t = 0; t < 4 && 4 * b + t < n; ++t) eps[4 * b + t] = (float)e[t];
+    normals4(block0 + nb, k0, k1, tab, e);
+#pragma unroll
+    for (uint32_t t = 0; t < 4; ++t) {
+      if (t < tail) {
+        const size_t i = 4 * (size_t)nb + t;
+        out[i] = RENOISE ? (float)fma(sigma, e[t], keep * (double)up[i]) : (float)e[t];
+      }
     }
   }
 }
 
-// x = (1 - sigma) up + sigma eps, blended in double from the unrounded eps
-// and rounded once to FP32.  x may alias up (each element is read before it
-// is written by the same thread), so neither pointer is restrict.
-__global__ void __launch_bounds__(kThreads, kBmBlocksPerSm) k_renoise(const float* up, float* x, int64_t n,
-                                                      double sigma, uint32_t k0, uint32_t k1, uint64_t block0) {
+__global__ void __launch_bounds__(kThreads, kBmBlocksPerSm)
+    k_philox_normal(float* __restrict__ eps, uint32_t nb, uint32_t tail, uint32_t k0, uint32_t k1, uint64_t block0) {
   __shared__ BmLogEntry s_log[LG_BM_LOG_ENTRIES];
   __shared__ BmTrigEntry s_trig[LG_BM_TRIG_ENTRIES];
   const BmTables tab = stage_bm_tables(s_log, s_trig);
-  const double keep = 1.0 - sigma;
-  const int64_t n_blocks = (n + 3) / 4;
-  for (int64_t b = gtid(); b < n_blocks; b += gstride()) {
-    double e[4];
-    normals4(block0 + (uint64_t)b, k0, k1, tab, e);
-    if (4 * b + 4 <= n) {
-      const float4 u = __ldcs(reinterpret_cast<const float4*>(up) + b);
-      float4 o;
-      o.x = (float)fma(sigma, e[0], keep * (double)u.x);
-      o.y = (float)fma(sigma, e[1], keep * (double)u.y);
-      o.z = (float)fma(sigma, e[2], keep * (double)u.z);
-      o.w = (float)fma(sigma, e[3], keep * (double)u.w);
-      __stcs(reinterpret_cast<float4*>(x) + b, o);
-    } else {
-      for (int t = 0; t < 4 && 4 * b + t < n; ++t) {
-        x[4 * b + t] = (float)fma(sigma, e[t], keep * (double)up[4 * b + t]);
-      }
-    }
-  }
+  normal_stream<false>(nullptr, eps, nb, tail, 0.0, k0, k1, block0, tab);
+}
+
+__global__ void __launch_bounds__(kThreads, kBmBlocksPerSm)
+    k_renoise(const float* up, float* x, uint32_t nb, uint32_t tail, double sigma, uint32_t k0, uint32_t k1,
+              uint64_t block0) {
+  __shared__ BmLogEntry s_log[LG_BM_LOG_ENTRIES];
+  __shared__ BmTrigEntry s_trig[LG_BM_TRIG_ENTRIES];
+  const BmTables tab = stage_bm_tables(s_log, s_trig);
+  normal_stream<true>(up, x, nb, tail, sigma, k0, k1, block0, tab);
 }
 
 // x += dt v with dt = sigma_next - sigma taken in FP32 (exact for the
@@ -202,18 +248,39 @@ cudaError_t launch_philox_u32(uint32_t* out, int64_t n_blocks, uint64_t seed, ui
   return cudaGetLastError();
 }
 
+// Normal stream / re-noise over n >= 1 elements starting at global element
+// 4 block0, in launches of at most 2^30 Philox blocks (32-bit indices inside).
+template <bool RENOISE>
+cudaError_t launch_normal_stream(const float* up, float* out, int64_t n, double sigma, uint64_t seed,
+                                 uint64_t block0, int sm_count, cudaStream_t s) {
+  constexpr int64_t kChunkBlocks = (int64_t)1 << 30;
+  const int64_t full = n / 4;
+  const uint32_t k0 = (uint32_t)seed, k1 = (uint32_t)(seed >> 32);
+  for (int64_t done = 0;;) {
+    const int64_t nb = std::min(full - done, kChunkBlocks);
+    const bool last = done + nb == full;
+    const uint32_t tail = last ? (uint32_t)(n % 4) : 0u;
+    const int grid = std::min(elementwise_grid(std::max<int64_t>(nb, 1), sm_count), kBmBlocksPerSm * sm_count);
+    if constexpr (RENOISE) {
+      k_renoise<<<grid, kThreads, 0, s>>>(up + 4 * done, out + 4 * done, (uint32_t)nb, tail, sigma, k0, k1,
+                                          block0 + (uint64_t)done);
+    } else {
+      k_philox_normal<<<grid, kThreads, 0, s>>>(out + 4 * done, (uint32_t)nb, tail, k0, k1, block0 + (uint64_t)done);
+    }
+    const cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess || last) return e;
+    done += nb;
+  }
+}
+
 cudaError_t launch_philox_normal(float* eps, int64_t n, uint64_t seed, uint64_t offset, int sm_count,
                                  cudaStream_t s) {
-  k_philox_normal<<<std::min(elementwise_grid((n + 3) / 4, sm_count), kBmBlocksPerSm * sm_count), kThreads, 0, s>>>(eps, n, (uint32_t)seed,
-                                                                               (uint32_t)(seed >> 32), offset / 4);
-  return cudaGetLastError();
+  return launch_normal_stream<false>(nullptr, eps, n, 0.0, seed, offset / 4, sm_count, s);
 }
 
 cudaError_t launch_renoise(const float* up, float* x, int64_t n, float sigma, uint64_t seed, uint64_t offset,
                            int sm_count, cudaStream_t s) {
-  k_renoise<<<std::min(elementwise_grid((n + 3) / 4, sm_count), kBmBlocksPerSm * sm_count), kThreads, 0, s>>>(up, x, n, (double)sigma, (uint32_t)seed,
-                                                                         (uint32_t)(seed >> 32), offset / 4);
-  return cudaGetLastError();
+  return launch_normal_stream<true>(up, x, n, (double)sigma, seed, offset / 4, sm_count, s);
 }
 
 cudaError_t launch_euler(float* x, const float* v, int64_t n, float dt, int sm_count, cudaStream_t s) {

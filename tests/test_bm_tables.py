@@ -3,9 +3,10 @@
 The committed include must be exactly what its generator writes, and the
 properties the device code relies on must hold: every 1/c_i has at most 28
 significant bits (so m * inv_c is exact for a 24-bit mantissa m), it is
-within 2^-27 of 1/c_i, the log entries are the logarithms they stand for,
-the trig entries are exact at quarter turns and on the unit circle.  Pure
-host work: no GPU, no oracle.
+within 2^-27 of 1/c_i, the log entries are -2 times the logarithms they
+stand for, the trig entries are exact at quarter turns, on the unit circle,
+and within a few double ulps (relative) of sin and cos evaluated with 40
+decimal digits, also next to the zeros.  Pure host work: no GPU, no oracle.
 """
 
 import importlib.util
@@ -13,6 +14,7 @@ import math
 import os
 import random
 import struct
+from decimal import Decimal, getcontext
 from fractions import Fraction
 
 import pytest
@@ -46,15 +48,16 @@ def test_committed_include_matches_generator():
 def test_log_table_invariants():
     rows = gen.log_table()
     assert len(rows) == 257
-    for i, (inv, L) in enumerate(rows):
+    for i, (inv, y) in enumerate(rows):
         c = 1.0 + i / 256.0
         assert _mantissa_bits_used(inv) <= 28
         assert abs(c * inv - 1.0) <= 2.0**-27
-        want = -math.log(2.0 * inv) if i > gen.LOG_SWITCH else -math.log(inv)
-        assert L == want
-        # the stored term never exceeds half of ln 2, so a nonzero multiple of
-        # ln 2 always dominates it
-        assert abs(L) <= 0.35
+        L = -math.log(2.0 * inv) if i > gen.LOG_SWITCH else -math.log(inv)
+        assert y == -2.0 * L  # exactly twice the double nearest the logarithm
+        # the stored term never exceeds ln 2 (half of the -2 ln 2 step), so a
+        # nonzero multiple of 2 ln 2 always dominates it
+        assert abs(y) <= 0.7
+        assert math.copysign(1.0, y) > 0 or y != 0.0  # no negative zero
     assert rows[0] == (1.0, 0.0) and rows[256] == (0.5, 0.0)
     # the switch sits at sqrt(2): the entries on either side straddle it
     assert 1 + gen.LOG_SWITCH / 256 < math.sqrt(2) < 1 + (gen.LOG_SWITCH + 1) / 256
@@ -77,23 +80,51 @@ def test_log_reduction_is_exact_for_every_mantissa_class():
             assert abs(r) <= Fraction(1, 512) + Fraction(1, 2**27)
 
 
+_PI40 = Decimal("3.141592653589793238462643383279502884197169")
+
+
+def _sincos40(i, n):
+    """sin and cos of 2 pi i / n by Taylor series with 40 significant digits."""
+    getcontext().prec = 45
+    a = 2 * _PI40 * i / n
+    a = a - (2 * _PI40) * int(a / (2 * _PI40))
+    s, c, term_s, term_c = Decimal(0), Decimal(0), a, Decimal(1)
+    for k in range(60):
+        s += term_s
+        c += term_c
+        term_s = -term_s * a * a / ((2 * k + 2) * (2 * k + 3))
+        term_c = -term_c * a * a / ((2 * k + 1) * (2 * k + 2))
+    return s, c
+
+
 def test_trig_table_invariants():
     rows = gen.trig_table()
-    assert len(rows) == 256
-    exact = {0: (0.0, 1.0), 64: (1.0, 0.0), 128: (0.0, -1.0), 192: (-1.0, 0.0)}
+    n = len(rows)
+    assert n == 1024
+    exact = {0: (0.0, 1.0), n // 4: (1.0, 0.0), n // 2: (0.0, -1.0), 3 * n // 4: (-1.0, 0.0)}
     for i, (s, c) in enumerate(rows):
         if i in exact:
             assert (s, c) == exact[i]
             assert math.copysign(1.0, s) > 0 or s != 0.0  # no negative zeros
             assert math.copysign(1.0, c) > 0 or c != 0.0
         assert abs(s * s + c * c - 1.0) <= 4e-16
-        a = 2 * math.pi * i / 256
+        a = 2 * math.pi * i / n
         assert abs(s - math.sin(a)) <= 1e-15 and abs(c - math.cos(a)) <= 1e-15
 
 
-@pytest.mark.parametrize("i", [1, 37, 64 + 5, 128 + 63, 255])
+@pytest.mark.parametrize("i", [1, 2, 127, 128, 129, 255, 257, 383, 511, 513, 700, 767, 769, 1022, 1023])
+def test_trig_entries_keep_relative_accuracy_next_to_zeros(i):
+    rows = gen.trig_table()
+    s40, c40 = _sincos40(i, len(rows))
+    s, c = rows[i]
+    assert abs((Decimal(s) - s40) / s40) <= Decimal(2.3e-16)
+    assert abs((Decimal(c) - c40) / c40) <= Decimal(2.3e-16)
+
+
+@pytest.mark.parametrize("i", [1, 37, 256 + 5, 512 + 255, 1023])
 def test_trig_table_symmetry(i):
     rows = gen.trig_table()
+    n = len(rows)
     s, c = rows[i]
-    s2, c2 = rows[(i + 64) % 256]  # a quarter turn later: (c, -s)
+    s2, c2 = rows[(i + n // 4) % n]  # a quarter turn later: (c, -s)
     assert (s2, c2) == (c + 0.0, -s + 0.0)
