@@ -237,3 +237,14 @@ def test_noalloc_reports_the_same_status_as_lg_lora_linear():
     assert L.lg_lora_linear_noalloc(x, W, A, B, y, 0, 32768, 32768, 576, None) == lg.LG_ERR_WORKSPACE
     assert L.lg_lora_linear(x, W, A, B, y, 0, 32768, 32768, 576, ws, lg.LG_NOALLOC_SCRATCH_BYTES, None) == \
         lg.LG_ERR_WORKSPACE
+
+
+
+def test_tuning_knobs_validate_their_range():
+    import lora_gemm_b200 as lg
+
+    L = lg.lib
+    for v in (3, 16, -1):
+        assert L.lg_set_cluster_size(v) == lg.LG_ERR_INVALID_ARG
+    for v in (-1, 3):
+        assert L.lg_set_kernel_variant(v) == lg.LG_ERR_INVALID_ARG
