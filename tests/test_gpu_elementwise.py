@@ -103,7 +103,7 @@ def test_renoise_in_place():
     assert torch.equal(up, ref)
 
 
-@pytest.mark.parametrize("name", ["tiny", "2k"])
+@pytest.mark.parametrize("name", ["tiny", "2k", "4k"])
 def test_euler_full_latent(name):
     w = synth.WORKLOADS[name]
     x = synth.upscaled_latent(w, DEV)
