@@ -108,7 +108,9 @@ constexpr uint32_t Y_STAGE_BYTES = 8 * Y_WARP_BYTES;              // 16 KiB for 
 template <bool PAIR, bool MX = false>
 struct Cfg {
   static constexpr int BN = PAIR ? 256 : 224;                         // output columns per tile
-  static constexpr uint32_t SF_COLS = MX ? 32u : 0u;                   // TMEM columns for MXFP8 scales
+  static constexpr int SF_BUFS = MX ? 4 : 0;                            // MXFP8 scale buffers in TMEM
+  static constexpr uint32_t SF_BUF_COLS = 16;                          // x 4 + W 2 x 4 columns, padded
+  static constexpr uint32_t SF_COLS = (uint32_t)SF_BUFS * SF_BUF_COLS;  // TMEM columns for MXFP8 scales
   static constexpr uint32_t SF_COL = TMEM_COLS - SF_COLS;              // first of them
   static constexpr uint32_t H_COL = (uint32_t)BN;                      // first TMEM column of h
   static constexpr int R_TMEM = (int)(TMEM_COLS - BN - SF_COLS) * 2;  // ranks of h held in TMEM
@@ -117,9 +119,19 @@ struct Cfg {
   static constexpr int HALF_N = BN / 2;                                // accumulator columns per epilogue warp
   static constexpr uint32_t B_ROWS = PAIR ? BN / 2 : BN;              // W / B_cat rows a CTA loads
   static constexpr uint32_t B_BYTES = B_ROWS * BK * 2;                // also 128 rows x 128 E4M3 codes
-  static constexpr uint32_t SF_OFF = A_BYTES + B_BYTES;               // MX: x scales, then 2 groups of W scales
-  static constexpr uint32_t STAGE = A_BYTES + B_BYTES + (MX ? 2048u : 0u);
+  static constexpr uint32_t STAGE = A_BYTES + B_BYTES;
+  // MX: the scales of a base-term stage (this CTA's x group, then both W
+  // groups) travel in a ring of their own, one slot per scale buffer.
+  static constexpr uint32_t SF_SLOT_BYTES = 2048;
+  static constexpr uint32_t SF_SLOTS_BYTES = MX ? (uint32_t)SF_BUFS * SF_SLOT_BYTES : 0u;
   static constexpr int MMA_M = PAIR ? 2 * BM : BM;
+  // Warps: producer, MMA, 8 epilogue warps, and for MXFP8 a warp that copies
+  // the scales of each stage into tensor memory ahead of the MMAs.
+  static constexpr int THREADS = MX ? NUM_THREADS + 32 : NUM_THREADS;
+  // y leaves through TMA stores from shared-memory boxes on SM pairs; the
+  // MXFP8 variant, whose shared memory holds a third tile of h instead,
+  // stores it straight from registers.
+  static constexpr bool Y_TMA = PAIR && !MX;
   static constexpr int PANEL = PAIR ? 2 * BM : BM;
   // Folded base term (narrow single-tile layers): its accumulator sits after
   // the widest down-projection chunk, below h.
@@ -130,7 +142,7 @@ struct Cfg {
   static_assert((PAIR ? HC_MAX / 2 : HC_MAX) * BK * 2 <= B_BYTES, "A_cat chunk tile must fit the B slot");
   static_assert(R_TMEM % BK == 0, "the TMEM / shared-memory split of h must fall on a K block");
   static_assert(HALF_N % 16 == 0 && HC_MAX <= BN, "epilogue and chunk widths");
-  static_assert(SF_COL + SF_COLS == TMEM_COLS && SF_OFF + (MX ? 2048u : 0u) == STAGE, "TMEM and stage layout");
+  static_assert(SF_COL + SF_COLS == TMEM_COLS && 3 * SF_GROUP_BYTES <= SF_SLOT_BYTES, "TMEM and scale layout");
 };
 
 struct Control {
@@ -142,6 +154,11 @@ struct Control {
   uint64_t slice_ready;        // every group member's slice of h is in its staging rows
   uint64_t slice_free;         // every group member has copied this CTA's slice
   uint64_t epi_sync;           // all epilogue warps finished writing this panel's h slice
+  uint64_t sfl_full[4];        // MXFP8: a scale slot's loads have landed (pair: counted on the leader)
+  uint64_t sfl_empty[4];       // MXFP8: a scale slot has been copied to TMEM and may be refilled
+  uint64_t sf_full[4];         // MXFP8: a TMEM scale buffer holds its stage's scales (leader)
+  uint64_t sf_empty[4];        // MXFP8: the MMAs that read a scale buffer are done (leader)
+  uint64_t sf_drain;           // MXFP8: every scale copy has finished (leader)
   uint32_t tmem_base;
   int abort_flag;
 };
@@ -166,6 +183,7 @@ struct Args {
   uint32_t control_off;     // byte offset of the Control block
   uint32_t h_tile_off;      // byte offset of the shared-memory tile of h (pair variant)
   uint32_t y_stage_off;     // byte offset of the y staging boxes (pair variant)
+  uint32_t sf_slot_off;     // byte offset of the MXFP8 scale slots
   // SwiGLU + MXFP8 output (MX variant, ffn > 0): W holds ffn gate rows then
   // ffn up rows; tile t covers gate rows [128 t, 128 t + 128) (leader CTA of
   // the pair) and the matching up rows (follower), and the epilogue writes
@@ -281,10 +299,15 @@ __device__ void run_producer(const CUtensorMap* tm_x, const CUtensorMap* tm_w, c
   // pair: y_n / 2 per CTA) after the A_cat chunk rows.
   const uint32_t wf_rows = PAIR ? (uint32_t)a.y_n / 2 : (uint32_t)a.y_n;
   const uint32_t tx_fold = tx_a + (a.fold ? mult * wf_rows * BK * 2 : 0u);
-  const uint32_t tx_k = mult * (A_BYTES + C::B_BYTES + (MX ? 3 * SF_GROUP_BYTES : 0u));
+  const uint32_t tx_k = mult * (A_BYTES + C::B_BYTES);
   const uint32_t tx_r = mult * C::B_BYTES;
+  const uint32_t tx_sf = mult * 3 * SF_GROUP_BYTES;
+  const uint32_t sfl_full_local = smem_u32(&ctl->sfl_full[0]);
+  const uint32_t sfl_full0 = PAIR ? mapa_shared(sfl_full_local, crank & ~1u) : sfl_full_local;
+  const uint32_t sfl_empty0 = smem_u32(&ctl->sfl_empty[0]);
   uint32_t stage = 0, phase = 0, sweep = 0, it = 0;
   uint64_t fills = 0;
+  uint32_t sf_fills = 0;  // MX: base-term stages whose scales were loaded
   bool ok = true;
   auto load = [&](const CUtensorMap* m, uint32_t dst, int c0, int c1) {
     if constexpr (PAIR) {
@@ -351,9 +374,22 @@ __device__ void run_producer(const CUtensorMap* tm_x, const CUtensorMap* tm_w, c
           const int nb1 = a.ffn > 0 ? a.ffn / BM + t : t * C::BN / BM + 1;  // ... and of rows 128-255
           load_x(tm_xq, sa, kb * BKQ, m0);
           load(tm_w, sa + A_BYTES, kb * BKQ, n0);
-          load(tm_sfa, sa + C::SF_OFF, 0, 2 * ((m0 / BM) * a.kq_blocks + kb));
-          load(tm_sfb, sa + C::SF_OFF + SF_GROUP_BYTES, 0, 2 * (nb0 * a.kq_blocks + kb));
-          load(tm_sfb, sa + C::SF_OFF + 2 * SF_GROUP_BYTES, 0, 2 * (nb1 * a.kq_blocks + kb));
+          // The scales into their own slot, once the scale-copy warp has
+          // moved the slot's previous contents to tensor memory.
+          const uint32_t b = sf_fills % (uint32_t)C::SF_BUFS;
+          if (!wait_bounded(sfl_empty0 + 8 * b, ((sf_fills / (uint32_t)C::SF_BUFS) & 1u) ^ 1u, a.wait_limit_ns,
+                            abort_flag)) {
+            ok = false;
+            ++fills;
+            advance(stage, phase, stages);
+            break;
+          }
+          const uint32_t slot = smem_base + a.sf_slot_off + b * C::SF_SLOT_BYTES;
+          if (posts_tx) mbar_arrive_expect_tx(sfl_full_local + 8 * b, tx_sf);
+          tma_load_2d_pair(slot, tm_sfa, sfl_full0 + 8 * b, 0, 2 * ((m0 / BM) * a.kq_blocks + kb));
+          tma_load_2d_pair(slot + SF_GROUP_BYTES, tm_sfb, sfl_full0 + 8 * b, 0, 2 * (nb0 * a.kq_blocks + kb));
+          tma_load_2d_pair(slot + 2 * SF_GROUP_BYTES, tm_sfb, sfl_full0 + 8 * b, 0, 2 * (nb1 * a.kq_blocks + kb));
+          ++sf_fills;
         } else {
           load_x(tm_x, sa, kb * BK, m0);
           load(tm_w, sa + A_BYTES, kb * BK, n0);
@@ -381,6 +417,10 @@ __device__ void run_producer(const CUtensorMap* tm_x, const CUtensorMap* tm_w, c
       const uint64_t fs = fills / stages + (s < fills % stages ? 1 : 0);
       if (fs) wait_teardown(full_local + 8 * s, (uint32_t)((fs - 1) & 1), abort_flag);
     }
+    for (uint32_t b = 0; MX && b < (uint32_t)C::SF_BUFS; ++b) {
+      const uint32_t fb = sf_fills / (uint32_t)C::SF_BUFS + (b < sf_fills % (uint32_t)C::SF_BUFS ? 1u : 0u);
+      if (fb) wait_teardown(sfl_full_local + 8 * b, (fb - 1) & 1u, abort_flag);
+    }
   } else if (!ok) {
     // A pair follower that gave up cannot observe the leader's barriers;
     // give its copies in flight (microseconds at most) time to land.
@@ -406,6 +446,8 @@ __device__ void run_mma(const Args& a, Control* ctl, uint32_t smem_base, uint32_
   const uint32_t empty0 = smem_u32(&ctl->empty[0]);
   const uint32_t acc_full = smem_u32(&ctl->acc_full);
   const uint32_t acc_empty = smem_u32(&ctl->acc_empty);
+  const uint32_t sf_full0 = smem_u32(&ctl->sf_full[0]);
+  const uint32_t sf_empty0 = smem_u32(&ctl->sf_empty[0]);
   const uint32_t idesc_h = idesc_bf16_f32(C::MMA_M, a.chunk_n);
   const uint32_t idesc_y = idesc_bf16_f32(C::MMA_M, a.y_n);
   const uint32_t d_acc = tmem + ACC_COL;
@@ -488,21 +530,26 @@ __device__ void run_mma(const Args& a, Control* ctl, uint32_t smem_base, uint32_
         const uint64_t da = sw128_kmajor_desc(sa);
         const uint64_t db = sw128_kmajor_desc(sa + A_BYTES);
         if constexpr (MX) {
-          // This stage's scales into one of two TMEM scale buffers (x rows in
-          // columns +0..3, W rows 0-127 in +4..7 and 128-255 in +8..11: row
-          // n's word sits in column n / 32), then four K = 32 MMAs, the k-th
-          // taking byte k of each row's scale word.  tcgen05.cp and
-          // tcgen05.mma of this thread run in issue order.
-          const uint32_t sf = tmem + C::SF_COL + 16u * (sf_buf & 1u);
-          ++sf_buf;
-          tmem_cp_32x128b_x4_pair(sf, plain_rows16_desc(sa + C::SF_OFF));
-          tmem_cp_32x128b_x4_pair(sf + 4, plain_rows16_desc(sa + C::SF_OFF + SF_GROUP_BYTES));
-          tmem_cp_32x128b_x4_pair(sf + 8, plain_rows16_desc(sa + C::SF_OFF + 2 * SF_GROUP_BYTES));
+          // The scale-copy warp has put this stage's scales into TMEM scale
+          // buffer sf_buf mod SF_BUFS (x rows in columns +0..3, W rows 0-127
+          // in +4..7 and 128-255 in +8..11: row n's word sits in column
+          // n / 32); once they are there, four K = 32 MMAs, the k-th taking
+          // byte k of each row's scale word, and the buffer goes back to the
+          // copy warp when they have completed.
+          const uint32_t b = sf_buf % (uint32_t)C::SF_BUFS;
+          if (!wait_bounded(sf_full0 + 8 * b, (sf_buf / (uint32_t)C::SF_BUFS) & 1u, a.wait_limit_ns, abort_flag)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t sf = tmem + C::SF_COL + C::SF_BUF_COLS * b;
 #pragma unroll
           for (int kk = 0; kk < BKQ / 32; ++kk) {
             umma_mx_pair(d_acc, da + 2 * kk, db + 2 * kk, idesc_mx_e4m3(C::MMA_M, C::BN, (uint32_t)kk, (uint32_t)kk),
                          sf, sf + 4, (i | kk) != 0);
           }
+          umma_commit_pair_mc(sf_empty0 + 8 * b, (uint16_t)(1u << crank));
+          ++sf_buf;
         } else {
 #pragma unroll
           for (int kk = 0; kk < BK / 16; ++kk) mma_ss(da + 2 * kk, db + 2 * kk, idesc_y, (i | kk) != 0);
@@ -542,6 +589,58 @@ __device__ void run_mma(const Args& a, Control* ctl, uint32_t smem_base, uint32_
   // Every MMA must finish before TMEM is freed or (for a pair) either CTA exits.
   commit(smem_u32(&ctl->drain));
   wait_teardown(smem_u32(&ctl->drain), 0, abort_flag);
+}
+
+// ---------------------------------------------------------------------------
+// Scale-copy warp (MXFP8, pair leader, one thread): for every base-term stage,
+// once its scales have landed in their slot and a TMEM scale buffer is free,
+// copies the three scale groups into that buffer (tcgen05.cp, both CTAs of
+// the pair, each from its own slot), then signals the MMA thread and hands
+// the slot back to both CTAs' producers.  Issued from a thread of its own,
+// the copies run beside the MMAs instead of between them; four slots and four
+// buffers let it work up to four stages ahead.  Its barriers count base-term
+// stages only, so it never waits on the operand ring.
+// ---------------------------------------------------------------------------
+template <bool PAIR, bool MX>
+__device__ void run_scale_copies(const Args& a, Control* ctl, uint32_t smem_base, uint32_t tmem, uint32_t crank,
+                                 uint32_t cid, uint32_t ncl, volatile int* abort_flag) {
+  if constexpr (MX) {
+    using C = Cfg<PAIR, MX>;
+    const int member = PAIR ? (int)(crank >> 1) : (int)crank;
+    const uint32_t sfl_full0 = smem_u32(&ctl->sfl_full[0]);
+    const uint32_t sfl_empty0 = smem_u32(&ctl->sfl_empty[0]);
+    const uint32_t sf_full0 = smem_u32(&ctl->sf_full[0]);
+    const uint32_t sf_empty0 = smem_u32(&ctl->sf_empty[0]);
+    const uint16_t self = (uint16_t)(1u << crank);
+    const uint16_t pair = (uint16_t)(3u << (crank & ~1u));
+    uint32_t n = 0;
+    bool ok = true;
+    const int kloop = a.fold ? 0 : a.kq_blocks;
+    for (int p = (int)cid; ok && p < a.num_panels; p += (int)ncl) {
+      for (int t = member; ok && t < a.n_tiles; t += a.group) {
+        for (int i = 0; i < kloop; ++i, ++n) {
+          const uint32_t b = n % (uint32_t)C::SF_BUFS;
+          const uint32_t q = (n / (uint32_t)C::SF_BUFS) & 1u;
+          if (!wait_bounded(sfl_full0 + 8 * b, q, a.wait_limit_ns, abort_flag) ||
+              !wait_bounded(sf_empty0 + 8 * b, q ^ 1u, a.wait_limit_ns, abort_flag)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t slot = smem_base + a.sf_slot_off + b * C::SF_SLOT_BYTES;
+          const uint32_t sf = tmem + C::SF_COL + C::SF_BUF_COLS * b;
+          tmem_cp_32x128b_x4_pair(sf, plain_rows16_desc(slot));
+          tmem_cp_32x128b_x4_pair(sf + 4, plain_rows16_desc(slot + SF_GROUP_BYTES));
+          tmem_cp_32x128b_x4_pair(sf + 8, plain_rows16_desc(slot + 2 * SF_GROUP_BYTES));
+          umma_commit_pair_mc(sf_full0 + 8 * b, self);
+          umma_commit_pair_mc(sfl_empty0 + 8 * b, pair);
+        }
+      }
+    }
+    // Every copy issued has finished before TMEM is freed.
+    umma_commit_pair_mc(smem_u32(&ctl->sf_drain), self);
+    wait_teardown(smem_u32(&ctl->sf_drain), 0, abort_flag);
+  }
 }
 
 // ---------------------------------------------------------------------------
@@ -904,7 +1003,7 @@ __device__ void run_epilogue(const CUtensorMap* tm_y, const Args& a, Control* ct
       release_acc(false);
 
       const int col0 = t * C::BN + half * C::HALF_N;
-      if constexpr (PAIR) {
+      if constexpr (C::Y_TMA) {
         // 32 x 32 boxes through this warp's staging buffer: convert, write
         // this lane's 64-byte row (16-byte chunk c at c ^ ((row / 2) mod 4),
         // the 64-byte swizzle), hand the box to a TMA store, and rewrite the
@@ -951,12 +1050,12 @@ __device__ void run_epilogue(const CUtensorMap* tm_y, const Args& a, Control* ct
     }
   }
   // The y stores of this warp have completed before the CTA can exit.
-  if (PAIR && lane == 0) bulk_wait_group0();
+  if (C::Y_TMA && lane == 0) bulk_wait_group0();
   __syncwarp();
 }
 
 template <bool PAIR, bool MX>
-__global__ void __launch_bounds__(NUM_THREADS, 1)
+__global__ void __launch_bounds__(Cfg<PAIR, MX>::THREADS, 1)
     k_lora_linear(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_w,
                   const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b,
                   const __grid_constant__ CUtensorMap tm_y, const __grid_constant__ CUtensorMap tm_xq,
@@ -986,11 +1085,18 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     mbar_init(smem_u32(&ctl->slice_ready), EPI_WARPS * args.group);
     mbar_init(smem_u32(&ctl->slice_free), EPI_WARPS * args.group);
     mbar_init(smem_u32(&ctl->epi_sync), EPI_WARPS);
+    for (int b = 0; b < 4; ++b) {
+      mbar_init(smem_u32(&ctl->sfl_full[b]), 1);
+      mbar_init(smem_u32(&ctl->sfl_empty[b]), 1);
+      mbar_init(smem_u32(&ctl->sf_full[b]), 1);
+      mbar_init(smem_u32(&ctl->sf_empty[b]), 1);
+    }
+    mbar_init(smem_u32(&ctl->sf_drain), 1);
     ctl->abort_flag = 0;
     fence_mbarrier_init();
     tma_prefetch_desc(&tm_x);
     tma_prefetch_desc(&tm_w);
-    if (PAIR) tma_prefetch_desc(&tm_y);
+    if (Cfg<PAIR, MX>::Y_TMA) tma_prefetch_desc(&tm_y);
     if (MX) {
       tma_prefetch_desc(&tm_xq);
       tma_prefetch_desc(&tm_sfa);
@@ -1025,6 +1131,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     __syncwarp();
   } else if (warp == 1) {
     if (lane == 0 && issues_mma) run_mma<PAIR, MX>(args, ctl, smem_base, tmem, crank, cid, ncl, abort_flag);
+    __syncwarp();
+  } else if (MX && warp == 2 + EPI_WARPS) {
+    if (lane == 0 && issues_mma) run_scale_copies<PAIR, MX>(args, ctl, smem_base, tmem, crank, cid, ncl, abort_flag);
     __syncwarp();
   } else {
     run_epilogue<PAIR, MX>(&tm_y, args, ctl, smem_base, tmem, crank, cid, ncl, warp, lane, abort_flag);
@@ -1125,7 +1234,7 @@ bool make_store_map(PFN_cuTensorMapEncodeTiled_v12000 enc, CUtensorMap* m, void*
 // shared memory goes to the ring.
 struct Geometry {
   int group = 1, slice = 0, n_chunks = 0, chunk_valid = 0, chunk_n = 16, stages = 0;
-  uint32_t staging_stride = 0, control_off = 0, h_tile_off = 0, y_stage_off = 0;
+  uint32_t staging_stride = 0, control_off = 0, h_tile_off = 0, y_stage_off = 0, sf_slot_off = 0;
   size_t smem = 0;
 };
 
@@ -1147,14 +1256,15 @@ bool make_geometry(int group, int R, Geometry* g) {
     if (C::H_SMEM && R > C::R_TMEM && (g->slice % 16 || g->chunk_valid % 16)) return false;
   }
   const uint32_t h_tile = (uint32_t)C::H_TILES * H_TILE_BYTES;
-  const uint32_t y_stage = PAIR ? Y_STAGE_BYTES : 0u;
-  const size_t fixed = 1024 + h_tile + y_stage + sizeof(Control);
+  const uint32_t y_stage = C::Y_TMA ? Y_STAGE_BYTES : 0u;
+  const size_t fixed = 1024 + h_tile + C::SF_SLOTS_BYTES + y_stage + sizeof(Control);
   g->stages = (int)((kMaxSmem - fixed) / C::STAGE);
   if (g->stages > MAX_STAGES) g->stages = MAX_STAGES;
   if (g->stages < 2) return false;
   if (group > 1 && (size_t)BM * g->staging_stride > (size_t)g->stages * C::STAGE) return false;
   g->h_tile_off = (uint32_t)g->stages * C::STAGE;  // 1024-aligned: stages are
-  g->y_stage_off = g->h_tile_off + h_tile;
+  g->sf_slot_off = g->h_tile_off + h_tile;
+  g->y_stage_off = g->sf_slot_off + C::SF_SLOTS_BYTES;
   g->control_off = g->y_stage_off + y_stage;
   g->smem = 1024 + (size_t)g->control_off + sizeof(Control);
   return true;
@@ -1165,7 +1275,8 @@ std::atomic<int> g_cluster_override{0};  // 0: automatic (lg_set_cluster_size)
 std::atomic<int> g_variant_override{0};  // 0: automatic, 1: single-SM MMA, 2: SM-pair MMA
 
 // Resident clusters of `cluster` CTAs of `kernel` on device `dev` (cached).
-int max_active_clusters(const void* kernel, int variant, int dev, int cluster, size_t smem, int sm_count) {
+int max_active_clusters(const void* kernel, int variant, int dev, int cluster, size_t smem, int sm_count,
+                        int threads) {
   static std::mutex mu;
   struct Entry {
     bool known = false;
@@ -1177,7 +1288,7 @@ int max_active_clusters(const void* kernel, int variant, int dev, int cluster, s
   if (en && en->known) return en->n;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3((unsigned)(cluster * sm_count), 1, 1);
-  cfg.blockDim = dim3(NUM_THREADS, 1, 1);
+  cfg.blockDim = dim3((unsigned)threads, 1, 1);
   cfg.dynamicSmemBytes = smem;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeClusterDimension;
@@ -1255,11 +1366,11 @@ cudaError_t launch_variant(const LinearLaunch& p, cudaStream_t s, int dev, int c
     tm_sfb = tm_x;
   }
   if (ok) {
-    if (PAIR && p.ffn == 0 && !p.eu_z) {
+    if (C::Y_TMA && p.ffn == 0 && !p.eu_z) {
       ok = make_store_map(enc, &tm_y, p.y, (uint64_t)p.N, (uint64_t)p.M);
     } else {
-      // Never used: the single-SM epilogue stores directly, SwiGLU writes
-      // MXFP8, the Euler output updates the latent.
+      // Never used: the single-SM and MXFP8 epilogues store directly, SwiGLU
+      // writes MXFP8, the Euler output updates the latent.
       tm_y = tm_x;
     }
   }
@@ -1303,16 +1414,17 @@ cudaError_t launch_variant(const LinearLaunch& p, cudaStream_t s, int dev, int c
   args.control_off = geo.control_off;
   args.h_tile_off = geo.h_tile_off;
   args.y_stage_off = geo.y_stage_off;
+  args.sf_slot_off = geo.sf_slot_off;
   args.wait_limit_ns = p.wait_limit_ns;
   const void* kernel = (const void*)k_lora_linear<PAIR, MX>;
-  int clusters = max_active_clusters(kernel, MX ? 3 : (PAIR ? 2 : 1), dev, cluster, geo.smem, p.sm_count);
+  int clusters = max_active_clusters(kernel, MX ? 3 : (PAIR ? 2 : 1), dev, cluster, geo.smem, p.sm_count, C::THREADS);
   if (clusters <= 0) clusters = p.sm_count / cluster;
   if (clusters > args.num_panels) clusters = args.num_panels;
   if (clusters < 1) clusters = 1;
 
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3((unsigned)(clusters * cluster), 1, 1);
-  cfg.blockDim = dim3(NUM_THREADS, 1, 1);
+  cfg.blockDim = dim3(C::THREADS, 1, 1);
   cfg.dynamicSmemBytes = geo.smem;
   cfg.stream = s;
   cudaLaunchAttribute attr[1];
