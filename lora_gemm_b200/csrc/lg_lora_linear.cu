@@ -32,13 +32,15 @@
 //   * Phase B (per N tile): a K loop x W^T into the accumulator, then R/16
 //     more MMAs with A = h read straight from TMEM (the last 64 ranks of the
 //     pair variant from the shared tile) and B = the B_cat tile; the epilogue
-//     converts the tile to bf16 and stores it (pairs: TMA stores).
+//     converts the tile to bf16 and stores it (bf16 pairs: TMA stores).
 //   * Warp roles: warp 0 issues TMA loads into a ring of stages of 64 K
 //     elements (128-byte swizzled K-major tiles: 44 KiB single-SM, 32 KiB per
 //     CTA of a pair), warp 1 issues the MMAs (one thread) and owns the TMEM
 //     allocation, warps 2-9 are the epilogue: each pulls half of the tile's
 //     accumulator into registers, releases the TMEM accumulator to the next
-//     tile's MMAs, then converts and stores y.
+//     tile's MMAs, then converts and stores y.  The MXFP8 variant adds warp
+//     10, which copies each stage's block scales into tensor memory ahead of
+//     the MMAs.
 //   * Output variants: bf16 y (the default); the FP32 latent updated in place
 //     by an Euler step (eu_z); MXFP8 codes and scales of silu(gate) * up
 //     (ffn, MXFP8 base term only).  A layer of one narrow tile (fold)
