@@ -823,7 +823,12 @@ def run_workloads(names, args, world, rank, dev, peaks):
     out = {}
     for name in names:
         w = synth.WORKLOADS[name]
-        P = Problem(w, dev, noise_offset=_dist().noise_offset(rank, w.latent_numel), lean=True)
+        if args.scaling == "strong":
+            frames = _dist().frame_shard(w.frames, rank, world)
+            _, (e0, _) = _dist().clip_shard(w.frames, w.channels, w.height, w.width, rank, world)
+            P = Problem(w, dev, noise_offset=e0, lean=True, frames=frames)
+        else:
+            P = Problem(w, dev, noise_offset=_dist().noise_offset(rank, w.latent_numel), lean=True)
         torch.cuda.synchronize()
         # Enough timed steps for >= 1.5 s under the clock sampler (200 ms period).
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -838,7 +843,8 @@ def run_workloads(names, args, world, rank, dev, peaks):
         kernels, flops, tflops = kernel_report(P, per, peaks)
         rec = {
             "latent": list(w.latent_shape), "tokens": P.M, "d": w.d, "layers_k_n": [list(x) for x in w.shapes],
-            "tokens_per_s": round(_dist().whole_job_rate(P.M, world, wargs.steps, ms), 1),
+            "tokens_per_s": round(w.tokens * wargs.steps / (ms * 1e-3) if args.scaling == "strong"
+                                  else _dist().whole_job_rate(P.M, world, wargs.steps, ms), 1),
             "ms_per_step": round(ms / wargs.steps, 3), "steps": wargs.steps, "warmup": args.warmup,
             "kernels": kernels, "clocks": clk, "gpu_launches": int(launches),
             "inputs": "lean: layer activations are views of one buffer of the widest K, outputs share one buffer",
