@@ -6,7 +6,7 @@ Usage: python lora_gemm_b200/build.py [--verbose]
 loads the library this script builds.)
 
 Compiles every csrc/*.cu with nvcc (-gencode arch=compute_100a,code=sm_100a,
--O3, -lineinfo, no fast-math), links them into one shared library next to
+-O3, -lineinfo, no fast-math, warnings as errors), links them into one shared library next to
 this file, and statically links the CUDA runtime so the library does not
 depend on the runtime version another package in the process loaded.
 """
@@ -26,7 +26,8 @@ LIB_NAME = "liblora_gemm.so"
 LIB_PATH = os.path.join(HERE, LIB_NAME)
 
 ARCH_FLAGS = ["-gencode", "arch=compute_100a,code=sm_100a"]
-COMMON_FLAGS = ["-std=c++17", "-O3", "-lineinfo", "-Xcompiler", "-fPIC", "-I", INCLUDE, "-I", CSRC]
+COMMON_FLAGS = ["-std=c++17", "-O3", "-lineinfo", "-Xcompiler", "-fPIC", "-Werror", "all-warnings", "-I", INCLUDE,
+                "-I", CSRC]
 
 
 def nvcc_path():

@@ -419,9 +419,11 @@ __device__ void run_producer(const CUtensorMap* tm_x, const CUtensorMap* tm_w, c
       const uint64_t fs = fills / stages + (s < fills % stages ? 1 : 0);
       if (fs) wait_teardown(full_local + 8 * s, (uint32_t)((fs - 1) & 1), abort_flag);
     }
-    for (uint32_t b = 0; MX && b < (uint32_t)C::SF_BUFS; ++b) {
-      const uint32_t fb = sf_fills / (uint32_t)C::SF_BUFS + (b < sf_fills % (uint32_t)C::SF_BUFS ? 1u : 0u);
-      if (fb) wait_teardown(sfl_full_local + 8 * b, (fb - 1) & 1u, abort_flag);
+    if constexpr (MX) {
+      for (uint32_t b = 0; b < (uint32_t)C::SF_BUFS; ++b) {
+        const uint32_t fb = sf_fills / (uint32_t)C::SF_BUFS + (b < sf_fills % (uint32_t)C::SF_BUFS ? 1u : 0u);
+        if (fb) wait_teardown(sfl_full_local + 8 * b, (fb - 1) & 1u, abort_flag);
+      }
     }
   } else if (!ok) {
     // A pair follower that gave up cannot observe the leader's barriers;
