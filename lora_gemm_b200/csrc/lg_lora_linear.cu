@@ -274,6 +274,36 @@ __device__ __forceinline__ void chunk_ranks(const Args& a, int member, int j, in
   count = max(0, min(a.chunk_valid, slice_end - first));
 }
 
+// The k-th work item of cluster cid: panel p and its N tiles [t0, t1).
+// Whole panels round-robin over the ncl clusters; when the last round holds
+// fewer panels than there are clusters, the idle clusters share them instead
+// of waiting: each panel of that round goes to the clusters c = j (mod
+// tail), which split its tiles (each such cluster computes the panel's h for
+// itself).  Every warp role walks the same list.
+struct Work {
+  int p, t0, t1;
+};
+__device__ __forceinline__ bool work_item(const Args& a, uint32_t cid, uint32_t ncl, int k, Work& w) {
+  const int n = (int)ncl, c = (int)cid;
+  const int full = a.num_panels / n;
+  if (k < full) {
+    w = Work{k * n + c, 0, a.n_tiles};
+    return true;
+  }
+  const int tail = a.num_panels - full * n;
+  if (k > full || tail == 0) return false;
+  if (a.n_tiles < 2) {  // nothing to split
+    if (c >= tail) return false;
+    w = Work{full * n + c, 0, a.n_tiles};
+    return true;
+  }
+  const int j = c % tail, q = c / tail;
+  const int shares = min((n - 1 - j) / tail + 1, a.n_tiles);  // clusters on panel j that get tiles
+  if (q >= shares) return false;
+  w = Work{full * n + j, q * a.n_tiles / shares, (q + 1) * a.n_tiles / shares};
+  return true;
+}
+
 // ---------------------------------------------------------------------------
 // Producer (warp 0, one thread): TMA loads into the stage ring.  The K sweep
 // alternates direction from one sweep to the next (serpentine order), so the
@@ -328,8 +358,9 @@ __device__ void run_producer(const CUtensorMap* tm_x, const CUtensorMap* tm_w, c
       tma_load_2d_hint(dst, m, full0 + 8 * stage, c0, c1, pol_x);
     }
   };
-  for (int p = (int)cid; ok && p < a.num_panels; p += (int)ncl, ++it) {
-    const int m0 = p * C::PANEL + half * BM;
+  Work w;
+  for (int k = 0; ok && work_item(a, cid, ncl, k, w); ++k, ++it) {
+    const int m0 = w.p * C::PANEL + half * BM;
     for (int j = 0; ok && j < a.n_chunks; ++j, ++sweep) {
       int first, count;
       chunk_ranks(a, member, j, first, count);
@@ -356,7 +387,7 @@ __device__ void run_producer(const CUtensorMap* tm_x, const CUtensorMap* tm_w, c
       ok = wait_bounded(slice_free, it & 1, a.wait_limit_ns, abort_flag, true);
       fence_proxy_async_smem();
     }
-    for (int t = member; ok && t < a.n_tiles; t += a.group, ++sweep) {
+    for (int t = w.t0 + member; ok && t < w.t1; t += a.group, ++sweep) {
       // A pair's MMA takes y_n / 2 B rows from each CTA (B_ROWS when y_n = BN).
       const int n0 = a.ffn > 0 ? (half ? a.ffn : 0) + t * BM : t * C::BN + half * (a.y_n / 2);
       const int kloop = a.fold ? 0 : (MX ? a.kq_blocks : a.k_blocks);
@@ -486,7 +517,8 @@ __device__ void run_mma(const Args& a, Control* ctl, uint32_t smem_base, uint32_
     }
   };
   const uint32_t a_rows = PAIR ? (uint32_t)a.chunk_n / 2 : (uint32_t)a.chunk_n;
-  for (int p = (int)cid; ok && p < a.num_panels; p += (int)ncl) {
+  Work w;
+  for (int k = 0; ok && work_item(a, cid, ncl, k, w); ++k) {
     for (int j = 0; ok && j < a.n_chunks; ++j) {
       if (!wait_bounded(acc_empty, acc_phase ^ 1, a.wait_limit_ns, abort_flag, PAIR)) {
         ok = false;
@@ -517,7 +549,7 @@ __device__ void run_mma(const Args& a, Control* ctl, uint32_t smem_base, uint32_
       commit(acc_full);
       acc_phase ^= 1;
     }
-    for (int t = member; ok && t < a.n_tiles; t += a.group) {
+    for (int t = w.t0 + member; ok && t < w.t1; t += a.group) {
       if (!wait_bounded(acc_empty, acc_phase ^ 1, a.wait_limit_ns, abort_flag, PAIR)) {
         ok = false;
         break;
@@ -620,8 +652,9 @@ __device__ void run_scale_copies(const Args& a, Control* ctl, uint32_t smem_base
     uint32_t n = 0;
     bool ok = true;
     const int kloop = a.fold ? 0 : a.kq_blocks;
-    for (int p = (int)cid; ok && p < a.num_panels; p += (int)ncl) {
-      for (int t = member; ok && t < a.n_tiles; t += a.group) {
+    Work w;
+    for (int k = 0; ok && work_item(a, cid, ncl, k, w); ++k) {
+      for (int t = w.t0 + member; ok && t < w.t1; t += a.group) {
         for (int i = 0; i < kloop; ++i, ++n) {
           const uint32_t b = n % (uint32_t)C::SF_BUFS;
           const uint32_t q = (n / (uint32_t)C::SF_BUFS) & 1u;
@@ -901,8 +934,9 @@ __device__ void run_epilogue(const CUtensorMap* tm_y, const Args& a, Control* ct
     }
     acc_phase ^= 1;
   };
-  for (int p = (int)cid; ok && p < a.num_panels; p += (int)ncl, ++it) {
-    const int64_t m0 = (int64_t)p * C::PANEL + parity * BM;
+  Work w;
+  for (int k = 0; ok && work_item(a, cid, ncl, k, w); ++k, ++it) {
+    const int64_t m0 = (int64_t)w.p * C::PANEL + parity * BM;
     for (int j = 0; ok && j < a.n_chunks; ++j) {
       ok = __all_sync(0xffffffffu, wait_bounded(acc_full, acc_phase, a.wait_limit_ns, abort_flag));
       if (!ok) break;
@@ -943,7 +977,7 @@ __device__ void run_epilogue(const CUtensorMap* tm_y, const Args& a, Control* ct
     }
     // The output tile's accumulator columns (folded base term: Y_FOLD_COL..).
     const uint32_t y_col = a.fold ? C::Y_FOLD_COL : ACC_COL;
-    for (int t = member; ok && t < a.n_tiles; t += a.group) {
+    for (int t = w.t0 + member; ok && t < w.t1; t += a.group) {
       ok = __all_sync(0xffffffffu, wait_bounded(acc_full, acc_phase, a.wait_limit_ns, abort_flag));
       if (!ok) break;
       tc_fence_after();
