@@ -1457,7 +1457,11 @@ cudaError_t launch_variant(const LinearLaunch& p, cudaStream_t s, int dev, int c
   const void* kernel = (const void*)k_lora_linear<PAIR, MX>;
   int clusters = max_active_clusters(kernel, MX ? 3 : (PAIR ? 2 : 1), dev, cluster, geo.smem, p.sm_count, C::THREADS);
   if (clusters <= 0) clusters = p.sm_count / cluster;
-  if (clusters > args.num_panels) clusters = args.num_panels;
+  // No more clusters than (panel, tile) pairs: with fewer panels than
+  // resident clusters the work list shares each panel's tiles among several
+  // clusters (each computing that panel's h).
+  const int64_t units = (int64_t)args.num_panels * (args.n_tiles >= 2 ? args.n_tiles : 1);
+  if (clusters > units) clusters = (int)units;
   if (clusters < 1) clusters = 1;
 
   cudaLaunchConfig_t cfg = {};
