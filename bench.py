@@ -823,12 +823,21 @@ def run_workloads(names, args, world, rank, dev, peaks):
     out = {}
     for name in names:
         w = synth.WORKLOADS[name]
-        if args.scaling == "strong":
-            frames = _dist().frame_shard(w.frames, rank, world)
-            _, (e0, _) = _dist().clip_shard(w.frames, w.channels, w.height, w.width, rank, world)
-            P = Problem(w, dev, noise_offset=e0, lean=True, frames=frames)
-        else:
-            P = Problem(w, dev, noise_offset=_dist().noise_offset(rank, w.latent_numel), lean=True)
+        # The inputs of a grid are allocated before anything is timed; a device
+        # without room for them (the 4K step holds ~123 GB) records that and
+        # moves on.  Every rank has the same device, so all ranks take the
+        # same branch and run the same collectives.
+        try:
+            if args.scaling == "strong":
+                frames = _dist().frame_shard(w.frames, rank, world)
+                _, (e0, _) = _dist().clip_shard(w.frames, w.channels, w.height, w.width, rank, world)
+                P = Problem(w, dev, noise_offset=e0, lean=True, frames=frames)
+            else:
+                P = Problem(w, dev, noise_offset=_dist().noise_offset(rank, w.latent_numel), lean=True)
+        except torch.cuda.OutOfMemoryError as e:
+            torch.cuda.empty_cache()
+            out[name] = {"unavailable": f"device memory: {str(e).splitlines()[0][:160]}"}
+            continue
         torch.cuda.synchronize()
         # Enough timed steps for >= 1.5 s under the clock sampler (200 ms period).
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
