@@ -80,13 +80,15 @@ __device__ __forceinline__ double hilo_to_double(uint32_t hi, uint32_t lo) {
 // multiple of ln 2 always dominates the table term (|ln u1| >= ln 2 - 0.35)
 // and no step cancels by more than a factor of two.
 __device__ __forceinline__ double neg2_ln_grid24(uint32_t n, const BmLogEntry* tab) {
-  const uint32_t lz = __clz(n);                             // 7..31 (kf = 31 - lz)
-  const uint32_t top = n << lz;                             // leading one at bit 31
-  const uint32_t i = (((top >> 22) + 1u) >> 1) - 256u;      // 0..256
+  // n <= 2^24 converts to FP32 exactly: its exponent field is kf + 127 and its
+  // 23 fraction bits are those of m = n 2^-kf.
+  const uint32_t fb = __float_as_uint(__uint2float_rn(n));
+  const uint32_t frac = fb & 0x7FFFFFu;
+  const uint32_t i = ((frac >> 14) + 1u) >> 1;              // nearest c_i = 1 + i/256: 0..256
   const BmLogEntry e = tab[i];
-  const uint32_t j = lz - 7u - (i > (uint32_t)kBmLogSwitch ? 1u : 0u);  // 24 - kf (- 1): 0..24
-  // m = n 2^-kf in [1, 2) from the bits of top (exact)
-  const double m = hilo_to_double(0x3FF00000u | ((top >> 11) & 0xFFFFFu), top << 21);
+  const uint32_t j = 151u - (fb >> 23) - (i > (uint32_t)kBmLogSwitch ? 1u : 0u);  // 24 - kf (- 1): 0..24
+  // m in [1, 2) from the fraction bits (exact)
+  const double m = hilo_to_double(0x3FF00000u | (frac >> 3), frac << 29);
   const double r = fma(m, e.inv_c, -1.0);
   double q = 1.0 / 3.0;
   q = fma(q, r, -2.0 / 5.0);
@@ -148,6 +150,14 @@ __device__ __forceinline__ void box_muller(uint32_t a, uint32_t b, const BmTable
   sincos_turn24(b >> 8, tab.trig, s, c);
   e_cos = rho * c;
   e_sin = rho * s;
+}
+
+// The radius and the angle of one pair of words (rho and cos, sin), for a
+// caller that scales rho once before using both products.
+__device__ __forceinline__ void box_muller_polar(uint32_t a, uint32_t b, const BmTables& tab, double& rho, double& c,
+                                                 double& s) {
+  rho = sqrt_seeded(neg2_ln_grid24((a >> 8) + 1u, tab.log));
+  sincos_turn24(b >> 8, tab.trig, s, c);
 }
 
 // ---------------------------------------------------------------------------

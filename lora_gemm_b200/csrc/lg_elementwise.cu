@@ -99,22 +99,33 @@ __device__ __forceinline__ void normal_stream(const float* up, float* out, uint3
     }
     // The U blocks are independent: their FP64 chains interleave.  A block
     // past nb is computed but not stored.
-    double e[U][4];
+    float4 o[U];
 #pragma unroll
-    for (int k = 0; k < U; ++k) normals4(block0 + b + k * stride, k0, k1, tab, e[k]);
+    for (int k = 0; k < U; ++k) {
+      const Words4 r = philox4x32_10(block0 + b + k * stride, k0, k1);
+      if constexpr (RENOISE) {
+        // sigma eps = (sigma rho) cos / sin: sigma scales the radius once
+        // per pair, each element then takes one fused multiply-add.
+        double rho, c, s;
+        box_muller_polar(r.w0, r.w1, tab, rho, c, s);
+        rho *= sigma;
+        o[k].x = (float)fma(rho, c, keep * (double)u[k].x);
+        o[k].y = (float)fma(rho, s, keep * (double)u[k].y);
+        box_muller_polar(r.w2, r.w3, tab, rho, c, s);
+        rho *= sigma;
+        o[k].z = (float)fma(rho, c, keep * (double)u[k].z);
+        o[k].w = (float)fma(rho, s, keep * (double)u[k].w);
+      } else {
+        double e[4];
+        box_muller(r.w0, r.w1, tab, e[0], e[1]);
+        box_muller(r.w2, r.w3, tab, e[2], e[3]);
+        o[k] = make_float4((float)e[0], (float)e[1], (float)e[2], (float)e[3]);
+      }
+    }
 #pragma unroll
     for (int k = 0; k < U; ++k) {
       if (k > 0 && b + k * stride >= nb) break;
-      float4 o;
-      if constexpr (RENOISE) {
-        o.x = (float)fma(sigma, e[k][0], keep * (double)u[k].x);
-        o.y = (float)fma(sigma, e[k][1], keep * (double)u[k].y);
-        o.z = (float)fma(sigma, e[k][2], keep * (double)u[k].z);
-        o.w = (float)fma(sigma, e[k][3], keep * (double)u[k].w);
-      } else {
-        o = make_float4((float)e[k][0], (float)e[k][1], (float)e[k][2], (float)e[k][3]);
-      }
-      __stcs(out4 + b + k * stride, o);
+      __stcs(out4 + b + k * stride, o[k]);
     }
   }
   if (tail && first == 0) {
