@@ -189,7 +189,7 @@ def set_wait_limit_ns(limit_ns):
 
 
 def set_cluster_size(g):
-    """SMs sharing one token panel in lora_linear (1, 2, 4, 8, 16; 0 = chosen per shape)."""
+    """SMs sharing one token panel in lora_linear (1, 2, 4, 8; 0 = chosen per shape)."""
     _check(lib.lg_set_cluster_size(int(g)), "lg_set_cluster_size")
 
 

@@ -49,22 +49,23 @@ __device__ __forceinline__ Words4 philox4x32_10(uint64_t block, uint32_t k0, uin
 // double and within a few double ulps of the exact values, so that the FP32
 // results (and any blend computed from them in double) round as the exact
 // values would.  Both uniforms are 24-bit integers scaled by 2^-24, which lets
-// every range reduction below be exact integer work; the two constant tables
+// every range reduction below be exact integer work; the three constant tables
 // come from gen_bm_tables.py and are staged in shared memory by the caller.
 // ---------------------------------------------------------------------------
-struct BmLogEntry {
+struct alignas(16) BmLogEntry {
   double inv_c;  // 1 / c_i cut to 28 significant bits, c_i = 1 + i / 256
   double y;      // -2 times the log term: 2 ln(inv_c), or 2 ln(2 inv_c) for i > LG_BM_LOG_SWITCH
 };
-struct BmTrigEntry {
-  double s, c;  // sin, cos of 2 pi i / 1024 (exact 0 and +-1 at quarter turns)
+struct alignas(16) BmTrigEntry {
+  double s, c;  // sin, cos of the entry's angle (exact 0 and +-1 at quarter turns)
 };
 struct BmTables {
-  const BmLogEntry* log;   // 257 entries
-  const BmTrigEntry* trig; // 1024 entries
+  const BmLogEntry* log;      // 257 entries
+  const BmTrigEntry* coarse;  // 4096 entries: 2 pi i / 4096
+  const BmTrigEntry* fine;    // 2049 entries: 2 pi k 2^-24, k = 0..2048
 };
 constexpr int kBmLogSwitch = 106;
-constexpr int kBmTrigBits = 10;  // 1024 trig entries
+constexpr int kBmCoarseBits = 12;  // 4096 coarse angles; the remainder takes the other 12 of 24 bits
 
 __device__ __forceinline__ double bits_to_double(uint64_t b) { return __longlong_as_double((long long)b); }
 __device__ __forceinline__ double hilo_to_double(uint32_t hi, uint32_t lo) {
@@ -74,11 +75,12 @@ __device__ __forceinline__ double hilo_to_double(uint32_t hi, uint32_t lo) {
 // y = -2 ln(n 2^-24) for an integer n in [1, 2^24] (Tang's table method).
 // With n = m 2^kf, m in [1, 2), the nearest grid point c_i = 1 + i/256 gives
 // r = m inv_c - 1 exactly (m has <= 24 significant bits, inv_c 28) and
-// |r| <= 2^-9 + 2^-27, so -2 log1p(r) = -2 r + r^2 q(r), q to the r^4 term
-// (the r^6 term of log1p), is within 2^-56 |r|.  Past c = sqrt 2 the entry
-// already holds the term of c/2 and the exponent is one higher, so a nonzero
-// multiple of ln 2 always dominates the table term (|ln u1| >= ln 2 - 0.35)
-// and no step cancels by more than a factor of two.
+// |r| <= 2^-9 + 2^-27, so -2 log1p(r) = r q(r), q the Horner form of
+// -2 + r - 2r^2/3 + r^3/2 - 2r^4/5 + r^5/3 (the log1p series to r^6), is
+// within 2^-56 |r|.  Past c = sqrt 2 the entry already holds the term of c/2
+// and the exponent is one higher, so a nonzero multiple of ln 2 always
+// dominates the table term (|ln u1| >= ln 2 - 0.35) and no step cancels by
+// more than a factor of two.
 __device__ __forceinline__ double neg2_ln_grid24(uint32_t n, const BmLogEntry* tab) {
   // n <= 2^24 converts to FP32 exactly: its exponent field is kf + 127 and its
   // 23 fraction bits are those of m = n 2^-kf.
@@ -95,15 +97,19 @@ __device__ __forceinline__ double neg2_ln_grid24(uint32_t n, const BmLogEntry* t
   q = fma(q, r, 1.0 / 2.0);
   q = fma(q, r, -2.0 / 3.0);
   q = fma(q, r, 1.0);
+  q = fma(q, r, -2.0);
   // (double)j from the bits of 2^52 + j
   const double jd = hilo_to_double(0x43300000u, j) - 0x1p52;
   const double base = fma(jd, 1.3862943611198906188, e.y);  // 2 j ln 2 + table term
-  return fma(r * r, q, fma(-2.0, r, base));
+  return fma(r, q, base);
 }
 
 // sqrt(y) for y = +-0 or y in [2^-24, 64): an FP32 reciprocal square root
-// seed, one Newton step on 1/sqrt(y) in double (relative error ~2^-44), then
-// one correction of y / sqrt(y) (error ~2^-88 before the final rounding).
+// seed r (relative error e, |e| < 2^-22 with the truncation of y to FP32),
+// then one third-order (Householder) step on sqrt(y) = t (1 - h)^(-1/2) with
+// t = y r and h = 1 - y r^2 = -2e - e^2: t (1 + h/2 + 3h^2/8) leaves a
+// truncation error of 5h^3/16 < 2^-64 relative, so the result is within
+// ~1.5 double ulps.
 __device__ __forceinline__ double sqrt_seeded(double y) {
   // max as signed: -0 (high word 0x80000000) takes the finite seed too
   const uint32_t hi = (uint32_t)max(__double2hiint(y), 0x3E700000);
@@ -111,43 +117,40 @@ __device__ __forceinline__ double sqrt_seeded(double y) {
   float rf;
   asm("rsqrt.approx.ftz.f32 %0, %1;" : "=f"(rf) : "f"(yf));
   const uint32_t rb = __float_as_uint(rf);
-  double r = hilo_to_double((rb >> 3) + (896u << 20), rb << 29);
+  const double r = hilo_to_double((rb >> 3) + (896u << 20), rb << 29);
   const double t = y * r;
-  const double hr = 0.5 * r;
-  r = fma(hr, fma(-t, r, 1.0), r);
-  const double s0 = y * r;
-  return fma(fma(-s0, s0, y), 0.5 * r, s0);
+  const double h = fma(-t, r, 1.0);
+  return fma(t * h, fma(h, 0.375, 0.5), t);
 }
 
-// sin and cos of 2 pi b 2^-24 for an integer b in [0, 2^24): the nearest
-// 1/1024 turn comes from the table, the remainder theta (|theta| <= pi/1024,
-// an exact integer rd times K = 2 pi 2^-24) from short Maclaurin series
-// (sin to theta^5, cos - 1 to theta^4: truncation below 2e-19 relative),
-// combined by the angle-addition formulas.  Near a zero of sin or cos the
-// table term is exactly zero, so the result keeps full relative accuracy.
-__device__ __forceinline__ void sincos_turn24(uint32_t b, const BmTrigEntry* tab, double& s, double& c) {
-  constexpr int kShift = 24 - kBmTrigBits;                   // 14
-  const uint32_t iu = ((b >> (kShift - 1)) + 1u) >> 1;       // nearest table point, 0..1024
-  // rd = b - iu 2^14 in [-2^13, 2^13), as a double from the bits of
-  // 2^52 + (rd + 2^13)
-  const uint32_t ri = b - (iu << kShift) + (1u << (kShift - 1));
-  const BmTrigEntry t = tab[iu & ((1u << kBmTrigBits) - 1u)];
-  const double rd = hilo_to_double(0x43300000u, ri) - (0x1p52 + 0x1p13);
-  constexpr double K = 6.283185307179586476925 * 0x1p-24;
-  constexpr double S3 = -K * K * K / 6.0, S5 = K * K * K * K * K / 120.0;
-  constexpr double C2 = -K * K / 2.0, C4 = K * K * K * K / 24.0;
-  const double z = rd * rd;                                  // exact (|rd| <= 2^13)
-  const double sth = rd * fma(z, fma(z, S5, S3), K);         // sin(theta)
-  const double cm1 = z * fma(z, C4, C2);                     // cos(theta) - 1
-  s = fma(t.s, cm1, fma(t.c, sth, t.s));
-  c = fma(t.c, cm1, fma(-t.s, sth, t.c));
+// sin and cos of 2 pi b 2^-24 for the integer b = w >> 8 of a 32-bit word w:
+// b = iu 2^12 + rd with iu the nearest 1/4096 turn and rd in [-2048, 2048),
+// both read off w by exact integer work, then the angle-addition formulas on
+// the coarse entry of iu and the fine entry of |rd| (sin negated for rd < 0).
+// Near a zero of sin or cos the coarse term is exactly zero, so the result
+// keeps full relative accuracy; elsewhere the angle is at least half a coarse
+// step from the zero, so each result is at least about half the larger of
+// its two products and the sum loses at most one bit.
+__device__ __forceinline__ void sincos_turn24(uint32_t w, const BmTables& tab, double& s, double& c) {
+  // (w + 2^19) >> 20 = (b + 2^11) >> 12 = iu; past the top it wraps to 0, the
+  // same angle.
+  const uint32_t iu = (w + (1u << 19)) >> 20;
+  // the low 12 bits of b, taken as a signed 12-bit integer, are rd
+  const uint32_t lo = w << 12;
+  const int rd = (int)lo >> 20;
+  const BmTrigEntry a = tab.coarse[iu];
+  const BmTrigEntry f = tab.fine[abs(rd)];
+  // sin of the remainder with the sign of rd (lo's sign bit)
+  const double sf = hilo_to_double((uint32_t)__double2hiint(f.s) ^ (lo & 0x80000000u), (uint32_t)__double2loint(f.s));
+  s = fma(a.s, f.c, a.c * sf);
+  c = fma(a.c, f.c, -(a.s * sf));
 }
 
 __device__ __forceinline__ void box_muller(uint32_t a, uint32_t b, const BmTables& tab, double& e_cos,
                                            double& e_sin) {
   const double rho = sqrt_seeded(neg2_ln_grid24((a >> 8) + 1u, tab.log));
   double s, c;
-  sincos_turn24(b >> 8, tab.trig, s, c);
+  sincos_turn24(b, tab, s, c);
   e_cos = rho * c;
   e_sin = rho * s;
 }
@@ -157,7 +160,7 @@ __device__ __forceinline__ void box_muller(uint32_t a, uint32_t b, const BmTable
 __device__ __forceinline__ void box_muller_polar(uint32_t a, uint32_t b, const BmTables& tab, double& rho, double& c,
                                                  double& s) {
   rho = sqrt_seeded(neg2_ln_grid24((a >> 8) + 1u, tab.log));
-  sincos_turn24(b >> 8, tab.trig, s, c);
+  sincos_turn24(b, tab, s, c);
 }
 
 // ---------------------------------------------------------------------------

@@ -9,6 +9,7 @@
 // dozens"; the merge follows "Open-H3-Regenerate-2K：MiniMax H3 的开源 4K
 // 精修方案", section "三个步如何完成工作".
 #include <algorithm>
+#include <mutex>
 
 #include "lg_bm_tables.inc"
 #include "lg_device.cuh"
@@ -19,26 +20,44 @@ namespace lg {
 namespace {
 
 constexpr int kThreads = 256;
-// The FP64 Box-Muller kernels are issue-bound.  On the 2K latent, with each
-// thread working on three Philox blocks at once (kBmUnroll), 2 blocks per SM
-// (122 registers a thread) gave 2.93 TB/s for the re-noise; one block at a
-// time gave 2.60 at 4 blocks per SM, two at a time 2.67-2.77 at 2-4.
-#ifndef LG_BM_BLOCKS_PER_SM
-#define LG_BM_BLOCKS_PER_SM 2
+// The FP64 Box-Muller kernels are issue-bound.  Each thread works on three
+// Philox blocks at once (kBmUnroll) so that their FP64 chains interleave; the
+// 100 KB of tables staged per block allow one 512-thread block per SM.
+#ifndef LG_BM_THREADS
+#define LG_BM_THREADS 512
 #endif
+#ifndef LG_BM_BLOCKS_PER_SM
+#define LG_BM_BLOCKS_PER_SM 1
+#endif
+constexpr int kBmThreads = LG_BM_THREADS;
 constexpr int kBmBlocksPerSm = LG_BM_BLOCKS_PER_SM;
 
 static_assert(LG_BM_LOG_SWITCH == kBmLogSwitch, "log table built for another switch point");
-__device__ const BmLogEntry g_bm_log[LG_BM_LOG_ENTRIES] = LG_BM_LOG_TABLE;
-__device__ const BmTrigEntry g_bm_trig[LG_BM_TRIG_ENTRIES] = LG_BM_TRIG_TABLE;
+static_assert(LG_BM_TRIG_COARSE_ENTRIES == 1 << kBmCoarseBits && LG_BM_TRIG_FINE_ENTRIES == (1 << (23 - kBmCoarseBits)) + 1,
+              "angle tables built for another split");
 
-// Copies the Box-Muller tables (8 KB) into the block's shared memory, where
-// the data-dependent lookups cost one shared load each.
-__device__ __forceinline__ BmTables stage_bm_tables(BmLogEntry* s_log, BmTrigEntry* s_trig) {
-  for (int i = threadIdx.x; i < LG_BM_LOG_ENTRIES; i += blockDim.x) s_log[i] = g_bm_log[i];
-  for (int i = threadIdx.x; i < LG_BM_TRIG_ENTRIES; i += blockDim.x) s_trig[i] = g_bm_trig[i];
+// The three tables in one image, copied to shared memory as 16-byte chunks.
+struct alignas(16) BmTableImage {
+  BmLogEntry log[LG_BM_LOG_ENTRIES];
+  BmTrigEntry coarse[LG_BM_TRIG_COARSE_ENTRIES];
+  BmTrigEntry fine[LG_BM_TRIG_FINE_ENTRIES];
+};
+static_assert(sizeof(BmTableImage) % 16 == 0, "table image is copied in 16-byte chunks");
+constexpr int kBmSmemBytes = (int)sizeof(BmTableImage);
+__device__ const BmTableImage g_bm_tables = {LG_BM_LOG_TABLE, LG_BM_TRIG_COARSE_TABLE, LG_BM_TRIG_FINE_TABLE};
+
+// Copies the Box-Muller tables into the block's (dynamic) shared memory with
+// asynchronous 16-byte copies, where the data-dependent lookups cost one
+// shared load each.
+__device__ __forceinline__ BmTables stage_bm_tables(uint8_t* smem) {
+  const uint8_t* src = reinterpret_cast<const uint8_t*>(&g_bm_tables);
+  const uint32_t dst = smem_u32(smem);
+  for (int i = threadIdx.x; i < kBmSmemBytes / 16; i += blockDim.x)
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst + 16 * i), "l"(src + 16 * i) : "memory");
+  asm volatile("cp.async.commit_group;\n\tcp.async.wait_all;" ::: "memory");
   __syncthreads();
-  return BmTables{s_log, s_trig};
+  const BmTableImage* t = reinterpret_cast<const BmTableImage*>(smem);
+  return BmTables{t->log, t->coarse, t->fine};
 }
 
 __device__ __forceinline__ int64_t gtid() { return (int64_t)blockIdx.x * blockDim.x + threadIdx.x; }
@@ -141,20 +160,18 @@ __device__ __forceinline__ void normal_stream(const float* up, float* out, uint3
   }
 }
 
-__global__ void __launch_bounds__(kThreads, kBmBlocksPerSm)
+__global__ void __launch_bounds__(kBmThreads, kBmBlocksPerSm)
     k_philox_normal(float* __restrict__ eps, uint32_t nb, uint32_t tail, uint32_t k0, uint32_t k1, uint64_t block0) {
-  __shared__ BmLogEntry s_log[LG_BM_LOG_ENTRIES];
-  __shared__ BmTrigEntry s_trig[LG_BM_TRIG_ENTRIES];
-  const BmTables tab = stage_bm_tables(s_log, s_trig);
+  extern __shared__ __align__(16) uint8_t bm_smem[];
+  const BmTables tab = stage_bm_tables(bm_smem);
   normal_stream<false>(nullptr, eps, nb, tail, 0.0, k0, k1, block0, tab);
 }
 
-__global__ void __launch_bounds__(kThreads, kBmBlocksPerSm)
+__global__ void __launch_bounds__(kBmThreads, kBmBlocksPerSm)
     k_renoise(const float* up, float* x, uint32_t nb, uint32_t tail, double sigma, uint32_t k0, uint32_t k1,
               uint64_t block0) {
-  __shared__ BmLogEntry s_log[LG_BM_LOG_ENTRIES];
-  __shared__ BmTrigEntry s_trig[LG_BM_TRIG_ENTRIES];
-  const BmTables tab = stage_bm_tables(s_log, s_trig);
+  extern __shared__ __align__(16) uint8_t bm_smem[];
+  const BmTables tab = stage_bm_tables(bm_smem);
   normal_stream<true>(up, x, nb, tail, sigma, k0, k1, block0, tab);
 }
 
@@ -259,24 +276,47 @@ cudaError_t launch_philox_u32(uint32_t* out, int64_t n_blocks, uint64_t seed, ui
   return cudaGetLastError();
 }
 
+// Lets the two Box-Muller kernels use the table image's dynamic shared
+// memory, once per CUDA context (the setting belongs to the context).
+cudaError_t configure_bm_kernels() {
+  static std::mutex mu;
+  static bool configured = false;
+  static unsigned long long context = 0;
+  std::lock_guard<std::mutex> lock(mu);
+  unsigned long long ctx = 0;
+  const bool have_ctx = current_context_id(&ctx);
+  if (have_ctx && configured && context == ctx) return cudaSuccess;
+  for (const void* k : {(const void*)k_renoise, (const void*)k_philox_normal}) {
+    const cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, kBmSmemBytes);
+    if (e != cudaSuccess) return e;
+  }
+  configured = have_ctx;
+  context = ctx;
+  return cudaSuccess;
+}
+
 // Normal stream / re-noise over n >= 1 elements starting at global element
 // 4 block0, in launches of at most 2^30 Philox blocks (32-bit indices inside).
 template <bool RENOISE>
 cudaError_t launch_normal_stream(const float* up, float* out, int64_t n, double sigma, uint64_t seed,
                                  uint64_t block0, int sm_count, cudaStream_t s) {
   constexpr int64_t kChunkBlocks = (int64_t)1 << 30;
+  const cudaError_t ce = configure_bm_kernels();
+  if (ce != cudaSuccess) return ce;
   const int64_t full = n / 4;
   const uint32_t k0 = (uint32_t)seed, k1 = (uint32_t)(seed >> 32);
   for (int64_t done = 0;;) {
     const int64_t nb = std::min(full - done, kChunkBlocks);
     const bool last = done + nb == full;
     const uint32_t tail = last ? (uint32_t)(n % 4) : 0u;
-    const int grid = std::min(elementwise_grid(std::max<int64_t>(nb, 1), sm_count), kBmBlocksPerSm * sm_count);
+    const int64_t want = (std::max<int64_t>(nb, 1) + kBmThreads - 1) / kBmThreads;
+    const int grid = (int)std::min<int64_t>(want, (int64_t)kBmBlocksPerSm * std::max(sm_count, 1));
     if constexpr (RENOISE) {
-      k_renoise<<<grid, kThreads, 0, s>>>(up + 4 * done, out + 4 * done, (uint32_t)nb, tail, sigma, k0, k1,
-                                          block0 + (uint64_t)done);
+      k_renoise<<<grid, kBmThreads, kBmSmemBytes, s>>>(up + 4 * done, out + 4 * done, (uint32_t)nb, tail, sigma, k0,
+                                                       k1, block0 + (uint64_t)done);
     } else {
-      k_philox_normal<<<grid, kThreads, 0, s>>>(out + 4 * done, (uint32_t)nb, tail, k0, k1, block0 + (uint64_t)done);
+      k_philox_normal<<<grid, kBmThreads, kBmSmemBytes, s>>>(out + 4 * done, (uint32_t)nb, tail, k0, k1,
+                                                             block0 + (uint64_t)done);
     }
     const cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess || last) return e;

@@ -4,9 +4,12 @@ The committed include must be exactly what its generator writes, and the
 properties the device code relies on must hold: every 1/c_i has at most 28
 significant bits (so m * inv_c is exact for a 24-bit mantissa m), it is
 within 2^-27 of 1/c_i, the log entries are -2 times the logarithms they
-stand for, the trig entries are exact at quarter turns, on the unit circle,
-and within a few double ulps (relative) of sin and cos evaluated with 40
-decimal digits, also next to the zeros.  Pure host work: no GPU, no oracle.
+stand for, the coarse angle entries are exact at quarter turns, every angle
+entry is on the unit circle and within half a double ulp (relative) of sin
+and cos evaluated with 40
+decimal digits, also next to the zeros; the two angle tables together give
+every 24-bit angle (exhaustively) within a few double ulps.  Pure host work:
+no GPU, no oracle.
 """
 
 import importlib.util
@@ -97,10 +100,10 @@ def _sincos40(i, n):
     return s, c
 
 
-def test_trig_table_invariants():
-    rows = gen.trig_table()
+def test_coarse_angle_table_invariants():
+    rows = gen.trig_coarse_table()
     n = len(rows)
-    assert n == 1024
+    assert n == 4096
     exact = {0: (0.0, 1.0), n // 4: (1.0, 0.0), n // 2: (0.0, -1.0), 3 * n // 4: (-1.0, 0.0)}
     for i, (s, c) in enumerate(rows):
         if i in exact:
@@ -112,19 +115,70 @@ def test_trig_table_invariants():
         assert abs(s - math.sin(a)) <= 1e-15 and abs(c - math.cos(a)) <= 1e-15
 
 
-@pytest.mark.parametrize("i", [1, 2, 127, 128, 129, 255, 257, 383, 511, 513, 700, 767, 769, 1022, 1023])
-def test_trig_entries_keep_relative_accuracy_next_to_zeros(i):
-    rows = gen.trig_table()
+def test_fine_angle_table_invariants():
+    rows = gen.trig_fine_table()
+    assert len(rows) == 2049 and rows[0] == (0.0, 1.0)
+    for k, (s, c) in enumerate(rows):
+        a = 2 * math.pi * k * 2.0**-24
+        assert 0.0 <= s <= a and c <= 1.0  # sin x <= x, cos x <= 1
+        assert abs(s - math.sin(a)) <= 1e-18 + 1e-15 * s and abs(c - math.cos(a)) <= 2.3e-16
+        assert abs(s * s + c * c - 1.0) <= 4e-16
+
+
+@pytest.mark.parametrize("i", [1, 2, 511, 512, 513, 1023, 1025, 1535, 2047, 2049, 3000, 3071, 3073, 4094, 4095])
+def test_coarse_entries_keep_relative_accuracy_next_to_zeros(i):
+    rows = gen.trig_coarse_table()
     s40, c40 = _sincos40(i, len(rows))
     s, c = rows[i]
-    assert abs((Decimal(s) - s40) / s40) <= Decimal(2.3e-16)
-    assert abs((Decimal(c) - c40) / c40) <= Decimal(2.3e-16)
+    assert abs((Decimal(s) - s40) / s40) <= Decimal(1.12e-16)
+    assert abs((Decimal(c) - c40) / c40) <= Decimal(1.12e-16)
 
 
-@pytest.mark.parametrize("i", [1, 37, 256 + 5, 512 + 255, 1023])
-def test_trig_table_symmetry(i):
-    rows = gen.trig_table()
+@pytest.mark.parametrize("k", [1, 2, 3, 100, 1000, 2047, 2048])
+def test_fine_entries_correctly_rounded(k):
+    s, c = gen.trig_fine_table()[k]
+    s40, c40 = _sincos40(k, 2**24)
+    assert abs((Decimal(s) - s40) / s40) <= Decimal(1.12e-16)
+    assert abs((Decimal(c) - c40) / c40) <= Decimal(1.12e-16)
+
+
+@pytest.mark.parametrize("i", [1, 37, 1024 + 5, 2048 + 1023, 4095])
+def test_coarse_table_symmetry(i):
+    rows = gen.trig_coarse_table()
     n = len(rows)
     s, c = rows[i]
     s2, c2 = rows[(i + n // 4) % n]  # a quarter turn later: (c, -s)
     assert (s2, c2) == (c + 0.0, -s + 0.0)
+
+
+def _two_level_sincos(b24):
+    """The device's angle split, in exact rational arithmetic on the table
+    entries, with each product and fused sum rounded to double as the device
+    rounds them: w = b24 << 8, iu = (w + 2^19) >> 20 mod 4096, rd = the low 12
+    bits of b24 as a signed integer."""
+    coarse, fine = gen.trig_coarse_table(), gen.trig_fine_table()
+    iu = ((b24 + 2048) >> 12) % 4096
+    rd = ((b24 & 4095) ^ 2048) - 2048
+    sa, ca = coarse[iu]
+    sb, cb = fine[abs(rd)]
+    sb = -sb if rd < 0 else sb
+    s = float(Fraction(sa) * Fraction(cb) + Fraction(ca * sb))
+    c = float(Fraction(ca) * Fraction(cb) - Fraction(sa * sb))
+    return s, c
+
+
+@pytest.mark.parametrize("b24", [0, 1, 2047, 2048, 2049, 4095, 4096, 4097, (1 << 22) - 2049, (1 << 22) - 2048,
+                                 (1 << 22) - 1, 1 << 22, (1 << 22) + 2047, (1 << 23) - 1, 1 << 23, (1 << 23) + 1,
+                                 (3 << 22) - 1, 3 << 22, (1 << 24) - 2049, (1 << 24) - 2048, (1 << 24) - 1,
+                                 0x5A5A5A, 0x123456, 0xABCDEF])
+def test_two_level_angles_near_zeros_and_splits(b24):
+    """Next to the zeros of sin and cos, at the split points of the remainder
+    and at the wrap of the coarse index, the two lookups give sin and cos of
+    2 pi b24 2^-24 within 4 double ulps (relative)."""
+    s, c = _two_level_sincos(b24)
+    s40, c40 = _sincos40(b24, 2**24)
+    for got, ref in ((s, s40), (c, c40)):
+        if abs(ref) < Decimal("1e-30"):  # an exact zero (the 40-digit series leaves ~1e-43)
+            assert got == 0.0
+        else:
+            assert abs((Decimal(got) - ref) / ref) <= Decimal(4 * 2.0**-53)
