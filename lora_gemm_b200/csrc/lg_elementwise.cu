@@ -48,13 +48,18 @@ __device__ const BmTableImage g_bm_tables = {LG_BM_LOG_TABLE, LG_BM_TRIG_COARSE_
 
 // Copies the Box-Muller tables into the block's (dynamic) shared memory with
 // asynchronous 16-byte copies, where the data-dependent lookups cost one
-// shared load each.
-__device__ __forceinline__ BmTables stage_bm_tables(uint8_t* smem) {
+// shared load each.  The copies are issued first and waited for later, so
+// the caller can issue its first global loads in between.
+__device__ __forceinline__ void stage_bm_tables_issue(uint8_t* smem) {
   const uint8_t* src = reinterpret_cast<const uint8_t*>(&g_bm_tables);
   const uint32_t dst = smem_u32(smem);
   for (int i = threadIdx.x; i < kBmSmemBytes / 16; i += blockDim.x)
     asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst + 16 * i), "l"(src + 16 * i) : "memory");
-  asm volatile("cp.async.commit_group;\n\tcp.async.wait_all;" ::: "memory");
+  asm volatile("cp.async.commit_group;" ::: "memory");
+}
+
+__device__ __forceinline__ BmTables stage_bm_tables_wait(const uint8_t* smem) {
+  asm volatile("cp.async.wait_all;" ::: "memory");
   __syncthreads();
   const BmTableImage* t = reinterpret_cast<const BmTableImage*>(smem);
   return BmTables{t->log, t->coarse, t->fine};
@@ -83,19 +88,50 @@ __device__ __forceinline__ void normals4(uint64_t block, uint32_t k0, uint32_t k
 // re-noise x = (1 - sigma) up + sigma eps (blended in double from the
 // unrounded eps and rounded once to FP32) over the elements [0, 4 nb + tail)
 // of one launch, whose element 0 is global element 4 block0.  Threads stride
-// over the nb full Philox blocks (one float4 each) with 32-bit indices; each
-// loads its next block of up before the FP64 work on the current one, so the
-// load's DRAM latency hides behind that work; the `tail` < 4 elements past
-// them go to thread 0 of block 0.  x may alias up (each element is read
-// before it is written by the same thread), so neither pointer is restrict.
+// over the nb full Philox blocks (one float4 each) with 32-bit indices, U
+// blocks at a time; each loads its next U blocks of up before the FP64 work
+// on the current ones, so the loads' DRAM latency hides behind that work.
+// The last, partial round computes only the blocks that exist, so the
+// threads that hold one block of it do a third of a round's work.  The
+// `tail` < 4 elements past the full blocks go to thread 0 of block 0.  x may
+// alias up (each element is read before it is written by the same thread),
+// so neither pointer is restrict.
 #ifndef LG_BM_UNROLL
 #define LG_BM_UNROLL 3
 #endif
 constexpr int kBmUnroll = LG_BM_UNROLL;  // Philox blocks a thread works on at once
 
+// One Philox block of the stream: 4 normals, or 4 re-noised elements of u.
+template <bool RENOISE>
+__device__ __forceinline__ float4 stream_block(uint64_t block, uint32_t k0, uint32_t k1, const BmTables& tab,
+                                               double sigma, double keep, const float4& u) {
+  const Words4 r = philox4x32_10(block, k0, k1);
+  float4 o;
+  if constexpr (RENOISE) {
+    // sigma eps = (sigma rho) cos / sin: sigma scales the radius once per
+    // pair, each element then takes one fused multiply-add.
+    double rho, c, s;
+    box_muller_polar(r.w0, r.w1, tab, rho, c, s);
+    rho *= sigma;
+    o.x = (float)fma(rho, c, keep * (double)u.x);
+    o.y = (float)fma(rho, s, keep * (double)u.y);
+    box_muller_polar(r.w2, r.w3, tab, rho, c, s);
+    rho *= sigma;
+    o.z = (float)fma(rho, c, keep * (double)u.z);
+    o.w = (float)fma(rho, s, keep * (double)u.w);
+  } else {
+    double e[4];
+    box_muller(r.w0, r.w1, tab, e[0], e[1]);
+    box_muller(r.w2, r.w3, tab, e[2], e[3]);
+    o = make_float4((float)e[0], (float)e[1], (float)e[2], (float)e[3]);
+  }
+  return o;
+}
+
 template <bool RENOISE>
 __device__ __forceinline__ void normal_stream(const float* up, float* out, uint32_t nb, uint32_t tail, double sigma,
-                                              uint32_t k0, uint32_t k1, uint64_t block0, const BmTables& tab) {
+                                              uint32_t k0, uint32_t k1, uint64_t block0, uint8_t* smem) {
+  stage_bm_tables_issue(smem);
   const double keep = 1.0 - sigma;
   const uint32_t stride = gridDim.x * blockDim.x;
   const uint32_t first = blockIdx.x * blockDim.x + threadIdx.x;
@@ -108,7 +144,10 @@ __device__ __forceinline__ void normal_stream(const float* up, float* out, uint3
     u_next[k] = make_float4(0.f, 0.f, 0.f, 0.f);
     if (RENOISE && first + k * stride < nb) u_next[k] = __ldcs(up4 + first + k * stride);
   }
-  for (uint32_t b = first; b < nb; b += U * stride) {
+  const BmTables tab = stage_bm_tables_wait(smem);
+  uint32_t b = first;
+  // Full rounds: all U blocks exist, and their FP64 chains interleave.
+  for (; b + (U - 1) * stride < nb; b += U * stride) {
     float4 u[U];
 #pragma unroll
     for (int k = 0; k < U; ++k) {
@@ -116,36 +155,18 @@ __device__ __forceinline__ void normal_stream(const float* up, float* out, uint3
       const uint32_t bn = b + (U + k) * stride;
       if (RENOISE && bn < nb) u_next[k] = __ldcs(up4 + bn);
     }
-    // The U blocks are independent: their FP64 chains interleave.  A block
-    // past nb is computed but not stored.
     float4 o[U];
 #pragma unroll
-    for (int k = 0; k < U; ++k) {
-      const Words4 r = philox4x32_10(block0 + b + k * stride, k0, k1);
-      if constexpr (RENOISE) {
-        // sigma eps = (sigma rho) cos / sin: sigma scales the radius once
-        // per pair, each element then takes one fused multiply-add.
-        double rho, c, s;
-        box_muller_polar(r.w0, r.w1, tab, rho, c, s);
-        rho *= sigma;
-        o[k].x = (float)fma(rho, c, keep * (double)u[k].x);
-        o[k].y = (float)fma(rho, s, keep * (double)u[k].y);
-        box_muller_polar(r.w2, r.w3, tab, rho, c, s);
-        rho *= sigma;
-        o[k].z = (float)fma(rho, c, keep * (double)u[k].z);
-        o[k].w = (float)fma(rho, s, keep * (double)u[k].w);
-      } else {
-        double e[4];
-        box_muller(r.w0, r.w1, tab, e[0], e[1]);
-        box_muller(r.w2, r.w3, tab, e[2], e[3]);
-        o[k] = make_float4((float)e[0], (float)e[1], (float)e[2], (float)e[3]);
-      }
-    }
+    for (int k = 0; k < U; ++k) o[k] = stream_block<RENOISE>(block0 + b + k * stride, k0, k1, tab, sigma, keep, u[k]);
 #pragma unroll
-    for (int k = 0; k < U; ++k) {
-      if (k > 0 && b + k * stride >= nb) break;
-      __stcs(out4 + b + k * stride, o[k]);
-    }
+    for (int k = 0; k < U; ++k) __stcs(out4 + b + k * stride, o[k]);
+  }
+  // The partial last round (up was prefetched for exactly these blocks).
+#pragma unroll
+  for (int k = 0; k < U; ++k) {
+    if (b + k * stride < nb)
+      __stcs(out4 + b + k * stride,
+             stream_block<RENOISE>(block0 + b + k * stride, k0, k1, tab, sigma, keep, u_next[k]));
   }
   if (tail && first == 0) {
     double e[4];
@@ -163,16 +184,14 @@ __device__ __forceinline__ void normal_stream(const float* up, float* out, uint3
 __global__ void __launch_bounds__(kBmThreads, kBmBlocksPerSm)
     k_philox_normal(float* __restrict__ eps, uint32_t nb, uint32_t tail, uint32_t k0, uint32_t k1, uint64_t block0) {
   extern __shared__ __align__(16) uint8_t bm_smem[];
-  const BmTables tab = stage_bm_tables(bm_smem);
-  normal_stream<false>(nullptr, eps, nb, tail, 0.0, k0, k1, block0, tab);
+  normal_stream<false>(nullptr, eps, nb, tail, 0.0, k0, k1, block0, bm_smem);
 }
 
 __global__ void __launch_bounds__(kBmThreads, kBmBlocksPerSm)
     k_renoise(const float* up, float* x, uint32_t nb, uint32_t tail, double sigma, uint32_t k0, uint32_t k1,
               uint64_t block0) {
   extern __shared__ __align__(16) uint8_t bm_smem[];
-  const BmTables tab = stage_bm_tables(bm_smem);
-  normal_stream<true>(up, x, nb, tail, sigma, k0, k1, block0, tab);
+  normal_stream<true>(up, x, nb, tail, sigma, k0, k1, block0, bm_smem);
 }
 
 // x += dt v with dt = sigma_next - sigma taken in FP32 (exact for the
