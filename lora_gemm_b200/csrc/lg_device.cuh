@@ -98,8 +98,7 @@ __device__ __forceinline__ double neg2_ln_grid24(uint32_t n, const BmLogEntry* t
   q = fma(q, r, -2.0 / 3.0);
   q = fma(q, r, 1.0);
   q = fma(q, r, -2.0);
-  // (double)j from the bits of 2^52 + j
-  const double jd = hilo_to_double(0x43300000u, j) - 0x1p52;
+  const double jd = __uint2double_rn(j);  // exact
   const double base = fma(jd, 1.3862943611198906188, e.y);  // 2 j ln 2 + table term
   return fma(r, q, base);
 }
