@@ -834,8 +834,10 @@ def run_workloads(names, args, world, rank, dev, peaks):
         w = synth.WORKLOADS[name]
         # The inputs of a grid are allocated before anything is timed; a device
         # without room for them (the 4K step holds ~123 GB) records that and
-        # moves on.  Every rank has the same device, so all ranks take the
-        # same branch and run the same collectives.
+        # moves on.  The ranks agree first (max over ranks of a failure flag),
+        # so that all of them skip the grid when any one is short of memory and
+        # every rank runs the same collectives.
+        P, err = None, None
         try:
             if args.scaling == "strong":
                 frames = _dist().frame_shard(w.frames, rank, world)
@@ -844,8 +846,11 @@ def run_workloads(names, args, world, rank, dev, peaks):
             else:
                 P = Problem(w, dev, noise_offset=_dist().noise_offset(rank, w.latent_numel), lean=True)
         except torch.cuda.OutOfMemoryError as e:
+            err = f"device memory: {str(e).splitlines()[0][:160]}"
+        if max_over_ranks(1.0 if err else 0.0, world) > 0.0:
+            del P
             torch.cuda.empty_cache()
-            out[name] = {"unavailable": f"device memory: {str(e).splitlines()[0][:160]}"}
+            out[name] = {"unavailable": err or "device memory on another rank"}
             continue
         torch.cuda.synchronize()
         # Enough timed steps for >= 1.5 s under the clock sampler (200 ms period).
