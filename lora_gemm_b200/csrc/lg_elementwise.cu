@@ -20,9 +20,10 @@ namespace lg {
 namespace {
 
 constexpr int kThreads = 256;
-// The FP64 Box-Muller kernels are issue-bound.  Each thread works on three
-// Philox blocks at once (kBmUnroll) so that their FP64 chains interleave; the
-// 100 KB of tables staged per block allow one 512-thread block per SM.
+// The FP64 Box-Muller kernels are bound by their mix of instructions and
+// shared-memory table gathers, not by HBM.  Each thread works on three Philox
+// blocks at once (kBmUnroll) so that their FP64 chains interleave; the 100 KB
+// of tables staged per block allow one 512-thread block per SM.
 #ifndef LG_BM_THREADS
 #define LG_BM_THREADS 512
 #endif
@@ -51,7 +52,7 @@ __device__ const BmTableImage g_bm_tables = {LG_BM_LOG_TABLE, LG_BM_TRIG_COARSE_
 // shared load each.  The copies are issued first and waited for later, so
 // the caller can issue its first global loads in between.
 __device__ __forceinline__ void stage_bm_tables_issue(uint8_t* smem) {
-  const uint8_t* src = reinterpret_cast<const uint8_t*>(&g_bm_tables);
+  const uint64_t src = (uint64_t)__cvta_generic_to_global(&g_bm_tables);
   const uint32_t dst = smem_u32(smem);
   for (int i = threadIdx.x; i < kBmSmemBytes / 16; i += blockDim.x)
     asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst + 16 * i), "l"(src + 16 * i) : "memory");
